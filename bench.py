@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the FP4 attention hot path on B200.
+
+One step = the whole hot path on one batch of synthetic input: the quantise
+prologue (smooth K + Hadamard + NVFP4 pack of Q and K) followed by the FP4
+attention forward, on the 15-second-clip workload (B=1, H=48, N=109568,
+d=128, non-causal).  Inputs are resident in HBM when timing starts; every
+input tensor (1.35 GB each) is larger than the 126 MB L2, so no flush is
+needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own replica
+of the workload (no data-path collective; weak scaling) and the time is the
+max over ranks.  ``--impl reference`` times the CPU oracle (as it stands) on
+the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_precision_b200 import synth  # noqa: E402
+
+METRIC = "FP4-attn TFLOPS @N=109k,d=128 (% composite roofline); quantize GB/s"
+UNIT = "TFLOP/s"
+WORKLOAD = "clip15s"
+PROLOGUE_BYTES_PER_ELEMENT = 5.125  # Q,K bf16 read (2+2) + codes (0.5+0.5) + scales (1/16+1/16)
+# ncu DRAM bytes (read + write) per launch of the attention kernel, keyed by
+# the sha256 of the attention source they were measured on; a changed kernel
+# reports null until it is profiled again.
+ATTN_TRAFFIC_BYTES = {}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def attention_flops(B, H, N, D=128):
+    return 4.0 * B * H * N * N * D
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def composite_peak(bf16_tflops):
+    """Peak of a contraction doing half its FLOPs on FP4 (4x the BF16 rate,
+    the nominal dense ratio) and half on BF16: 2 / (1/P_fp4 + 1/P_bf16)."""
+    p4 = 4.0 * bf16_tflops
+    return 2.0 / (1.0 / p4 + 1.0 / bf16_tflops)
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.strip().split(", ") for r in self.file.read().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 10:
+                continue
+            try:
+                sm.append(float(r[2]))
+                mx.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[6:10]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed ----
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------- CPU baseline -----
+
+def cpu_sample(w, target_s=12.0, max_rows=4096):
+    """Time the oracle (as it stands) on one head of the workload: its prologue
+    and the attention of R query rows against all N keys, R sized for about
+    target_s seconds.  Returns dict with TFLOP/s of the attention sample."""
+    import oracle
+    d = synth.generate(w, ("q", "k", "v"), heads=[0])
+    qb, kb, vb = (synth.bf16_bits(d[t]) for t in "qkv")
+    t0 = time.perf_counter()
+    codes = oracle.quantize_qk(qb, kb)
+    t_pro = time.perf_counter() - t0
+    qh = oracle.dequant(codes["q_codes"][0, 0], codes["q_scales"][0, 0])
+    kh = oracle.dequant(codes["k_codes"][0, 0], codes["k_scales"][0, 0])
+    rows = synth.sample_rows(w.N, 32, seed=w.seed)
+    t0 = time.perf_counter()
+    oracle.attention_head(qh, kh, vb[0, 0], rows=rows)
+    t_probe = time.perf_counter() - t0
+    R = int(min(max_rows, max(32, 32 * target_s / max(t_probe, 1e-3))))
+    rows = synth.sample_rows(w.N, R, seed=w.seed)
+    t0 = time.perf_counter()
+    oracle.attention_head(qh, kh, vb[0, 0], rows=rows)
+    t_att = time.perf_counter() - t0
+    flops = 4.0 * R * w.N * 128
+    return dict(value=flops / t_att / 1e12, unit=UNIT, cores=oracle.num_threads(), kind="oracle",
+                sample=(f"head 0 of {w.name}: fp64 attention of {R} query rows against all {w.N} keys "
+                        f"({t_att:.1f} s); oracle prologue of that head's Q and K took {t_pro:.2f} s "
+                        f"({PROLOGUE_BYTES_PER_ELEMENT * w.N * 128 / t_pro / 1e9:.3f} GB/s)"),
+                prologue_gbs=PROLOGUE_BYTES_PER_ELEMENT * w.N * 128 / t_pro / 1e9)
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: each step is a bounded sample of the workload on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    d = synth.generate(w, ("q", "k", "v"), heads=[0])
+    qb, kb, vb = (synth.bf16_bits(d[t]) for t in "qkv")
+    codes = oracle.quantize_qk(qb, kb)
+    qh = oracle.dequant(codes["q_codes"][0, 0], codes["q_scales"][0, 0])
+    kh = oracle.dequant(codes["k_codes"][0, 0], codes["k_scales"][0, 0])
+    R = args.ref_rows
+    rows = synth.sample_rows(w.N, R, seed=w.seed)
+
+    def step():
+        c = oracle.quantize_qk(qb[:, :, :4096], kb[:, :, :4096])  # prologue on a slice of the head
+        oracle.attention_head(qh, kh, vb[0, 0], rows=rows)
+        return c
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 4.0 * R * w.N * 128
+    value = flops / dt / 1e12
+    sample = (f"per step: oracle prologue of 4096 rows of head 0 plus fp64 attention of {R} query rows of "
+              f"head 0 of {w.name} against all {w.N} keys")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": 128, "causal": False,
+                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- our arm ------
+
+def run_ours(args, rank, world, local):
+    from nvfp4_precision_b200 import fp4attn as fa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    B, H, N = w.B, w.H, w.N
+    t0 = time.perf_counter()
+    host = synth.generate(w)
+    log(f"[rank {rank}] inputs generated in {time.perf_counter() - t0:.1f} s: {w.describe()}")
+    q, k, v = (host[t].to(dev) for t in "qkv")
+    out = dict(q_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
+               q_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
+               k_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
+               k_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
+               k_mean=torch.empty((B, H, 128), dtype=torch.float32, device=dev))
+    o = torch.empty_like(v)
+    ws = fa.new_workspace(B, H, N, dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 3  # key sums, quantise, attention
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fp4attn_quantize_qk(q, k, flags=0, out=out, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        fa.fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, o=o,
+                           workspace=ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = fa.fp4attn_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {fa.status_string(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local) if not args.no_clocks else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    barrier(world)
+    ms_step = start.elapsed_time(end) / args.steps
+    ms_pro = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_step_max = max_over_ranks(ms_step, world, dev)
+    ms_pro_max = max_over_ranks(ms_pro, world, dev)
+    ms_att_max = max_over_ranks(ms_att, world, dev)
+    st = fa.fp4attn_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {fa.status_string(st)}")
+
+    F = attention_flops(B, H, N)
+    value = world * F / (ms_step_max * 1e-3) / 1e12
+    peaks = measured_peaks()
+    p_comp = composite_peak(peaks["bf16_sustained"])
+    att_tflops = F / (ms_att_max * 1e-3) / 1e12
+    pro_bytes = PROLOGUE_BYTES_PER_ELEMENT * B * H * N * 128
+    pro_gbs = pro_bytes / (ms_pro_max * 1e-3) / 1e9
+    att_src = os.path.join(ROOT, "nvfp4_precision_b200", "csrc", "attention.cu")
+    traffic = ATTN_TRAFFIC_BYTES.get(source_hash(att_src))
+
+    # ---- end to end through the public API: pinned host inputs in, O out ----
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (host[t].pin_memory() for t in "qkv")
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = max_over_ranks(s2.elapsed_time(e2) / args.e2e_steps, world, dev)
+        e2e = {"value": world * F / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(q.numel() * 2 * 3), "d2h_bytes_per_step": int(o.numel() * 2),
+               "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_sample(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp4(e2m1,ue4m3)xbf16->f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": 128, "causal": False,
+                       "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (no flush needed)",
+                       "step": "quantize prologue + attention forward"},
+            "attention": {"ms": ms_att_max, "tflops": att_tflops,
+                          "frac_composite_sustained": att_tflops / p_comp,
+                          "frac_composite_nominal": att_tflops / composite_peak(2250.0)},
+            "quantize": {"ms": ms_pro_max, "gbs": pro_gbs, "frac_hbm": pro_gbs / peaks["hbm_gbs"],
+                         "bytes": pro_bytes},
+            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": p_comp, "unit": "TFLOP/s",
+                         "frac": att_tflops / p_comp, "traffic": traffic,
+                         "peak_note": (f"composite FP4/BF16 peak from {peaks['source']} sustained bf16 "
+                                       f"{peaks['bf16_sustained']} TFLOP/s x nominal FP4:BF16 ratio 4")},
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        # the oracle arm runs on rank 0's host cores only; other ranks exit at once
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_reference(args, 0, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_init()
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * fp4attn -- FP4 dense attention for long non-causal sequences on NVIDIA B200.
+ *
+ * C ABI of the CUDA library (nvfp4_precision_b200/libfp4attn.so).  Plain
+ * pointers and sizes only; every call is stream-ordered and asynchronous
+ * unless stated otherwise.  The library allocates no memory and keeps no
+ * state between calls: the caller owns every buffer, including the small
+ * workspace that holds the device-side status word and the key-mean sums.
+ *
+ * The method (FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention"):
+ *   1. smooth K: subtract each head's mean key (exact for softmax, since
+ *      q.(k_j - kbar) = q.k_j - q.kbar is a shift shared by every key);
+ *   2. rotate Q and K by the same orthonormal 128x128 Hadamard matrix (exact,
+ *      since (qH).(kH) = q.k; spreads outlier channels across scale blocks);
+ *   3. quantise Q and K to NVFP4: E2M1 values with one E4M3 scale per 16
+ *      channels under an fp32 per-tensor scale (unit by default);
+ *   4. softmax(Q K^T * scale) V with Q K^T from the FP4 operands and P, V in
+ *      BF16, non-causal, dense.
+ * Details the pages leave open are fixed as follows: block scale amax/6,
+ * round-to-nearest-even with saturation for both formats, Sylvester-ordered
+ * Hadamard applied as seven fp32 butterfly stages of ascending stride followed
+ * by one multiply by fp32(1/sqrt(128)), and an exact int64 fixed-point key sum
+ * (2^-24 resolution) so the mean does not depend on summation order.
+ *
+ * Layouts (all tensors contiguous, row-major, head dim D = 128):
+ *   Q, K, V      bf16  [B, H, N, 128]
+ *   codes        uint8 [B, H, N, 64]   element 2i in the low nibble of byte i;
+ *                                      sign in bit 3 of each nibble
+ *   scales       uint8 [B, H, N, 8]    UE4M3 scale of channels 16j..16j+15
+ *   k_mean       fp32  [B, H, 128]
+ *   O            bf16  [B, H, N, 128]
+ *   lse          fp32  [B, H, N]       natural-log sum of exp of the scaled logits
+ * Every pointer must be 16-byte aligned.  Pointers named *_dev are device
+ * pointers (cudaMalloc / torch CUDA tensors); none may alias another output.
+ *
+ * Error behaviour: argument errors are returned synchronously and nothing is
+ * launched.  A failed launch returns FP4ATTN_ERR_CUDA (the CUDA error is
+ * cleared).  Errors found on the device (non-finite or out-of-range input,
+ * a bounded wait that ran out) are written to the workspace status word and
+ * read with fp4attn_read_status.  No call exits the process or traps.
+ */
+#ifndef FP4ATTN_H
+#define FP4ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4ATTN_OK = 0,
+    FP4ATTN_ERR_INVALID_ARG = 1,  /* bad shape, NULL or misaligned pointer      */
+    FP4ATTN_ERR_UNSUPPORTED = 2,  /* valid but not supported (e.g. D != 128)    */
+    FP4ATTN_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed          */
+    FP4ATTN_ERR_RANGE = 4,        /* device: non-finite input, |k| >= 2^20, g<=0 */
+    FP4ATTN_ERR_TIMEOUT = 5,      /* device: a bounded wait ran out             */
+    FP4ATTN_ERR_WORKSPACE = 6     /* workspace missing or too small             */
+} fp4attn_status;
+
+/* Flags of fp4attn_quantize_qk (0 = the full method).  Both exist for
+ * ablation and for checking the quantiser on its own. */
+enum {
+    FP4ATTN_NO_SMOOTH_K = 1u,  /* do not subtract the key mean (k_mean reports 0) */
+    FP4ATTN_NO_HADAMARD = 2u   /* do not rotate Q and K                           */
+};
+
+typedef struct {
+    int32_t B, H, N, D;  /* D must be 128; B, H, N >= 0; N <= 262144 */
+} fp4attn_shape;
+
+/* Bytes of workspace that fp4attn_quantize_qk and fp4attn_forward need for
+ * this shape (status word, per-head int64 key sums).  Never 0. */
+size_t fp4attn_workspace_bytes(fp4attn_shape s);
+
+/* Smooth K + Hadamard + NVFP4 pack of Q and K (method steps 1-3).
+ *   q_bf16_dev, k_bf16_dev : [B,H,N,128] bf16 inputs.
+ *   q_gscale_dev, k_gscale_dev : device fp32 scalars g (finite, > 0), or NULL
+ *     for 1.0.  Block scale s = UE4M3(amax / 6 / g); the value of a code is
+ *     g * s * e2m1.
+ *   flags : FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD, or 0.
+ *   q_codes_dev, k_codes_dev : [B,H,N,64] out.  q_scales_dev, k_scales_dev :
+ *     [B,H,N,8] out.  k_mean_dev : [B,H,128] fp32 out, or NULL.
+ *   workspace_dev : fp4attn_workspace_bytes(s) bytes; cleared by this call.
+ * Device errors: FP4ATTN_ERR_RANGE for a non-finite Q or K value, |k| >= 2^20
+ * (the key sum would leave its exact range) or g not finite and > 0; the
+ * affected outputs are unspecified. */
+int fp4attn_quantize_qk(const void* q_bf16_dev, const void* k_bf16_dev, fp4attn_shape s,
+                        const float* q_gscale_dev, const float* k_gscale_dev, uint32_t flags,
+                        uint8_t* q_codes_dev, uint8_t* q_scales_dev,
+                        uint8_t* k_codes_dev, uint8_t* k_scales_dev, float* k_mean_dev,
+                        void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
+
+/* Non-causal attention over NVFP4 Q and K and bf16 V (method step 4):
+ *   O = softmax(scale * gQ * gK * (Qc K c^T)) V,  Qc, Kc the block-scaled E2M1
+ *   values; Q K^T on the FP4 tensor cores with fp32 accumulation, P rounded to
+ *   bf16 for P.V, fp32 accumulation, online softmax.
+ *   softmax_scale : <= 0 selects 1/sqrt(128).
+ *   o_bf16_dev : [B,H,N,128] out.  lse_dev : [B,H,N] out or NULL.
+ *   workspace_dev : as for fp4attn_quantize_qk (status word only; not cleared).
+ * Device errors: FP4ATTN_ERR_RANGE for a bad g; FP4ATTN_ERR_TIMEOUT if an
+ * internal wait ran out (the output is then incomplete). */
+int fp4attn_forward(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
+                    const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                    const float* q_gscale_dev, const float* k_gscale_dev,
+                    const void* v_bf16_dev, fp4attn_shape s, float softmax_scale,
+                    void* o_bf16_dev, float* lse_dev,
+                    void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
+
+/* Testing: decode NVFP4 rows back to fp32, out = fl(fl(g * s) * e2m1).
+ *   codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or NULL,
+ *   out_dev fp32 [rows,128], rows = B*H*N of s. */
+int fp4attn_dequant(const uint8_t* codes_dev, const uint8_t* scales_dev, const float* gscale_dev,
+                    fp4attn_shape s, float* out_dev, cudaStream_t stream);
+
+/* Read (synchronously: waits for the stream) and return in *device_status the
+ * workspace status word: FP4ATTN_OK or the first device error. */
+int fp4attn_read_status(const void* workspace_dev, cudaStream_t stream, int* device_status);
+
+/* Reset the workspace status word to FP4ATTN_OK (stream-ordered). */
+int fp4attn_reset_status(void* workspace_dev, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* fp4attn_status_string(int code);
+
+/* ---- test hooks: the same device building blocks, exposed for unit tests ---- */
+
+/* Element-wise fp32 -> E2M1 code (low nibble; sign in bit 3) and -> E4M3 byte
+ * with the device conversions the quantiser uses (round to nearest even,
+ * saturating).  n elements; either output may be NULL. */
+int fp4attn_encode_f32(const float* x_dev, int64_t n, uint8_t* e2m1_dev, uint8_t* e4m3_dev,
+                       cudaStream_t stream);
+
+/* One 128x128 tile of raw FP4 scores S = Qc . Kc^T (fp32, no softmax scale,
+ * no global scales) through the same tcgen05 block-scaled MMA, scale-factor
+ * staging and descriptors as fp4attn_forward.  q_* and k_* point at the
+ * first of 128 rows (codes [128,64], scales [128,8]); s_out_dev fp32 [128,128]. */
+int fp4attn_probe_qk_tile(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
+                          const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                          float* s_out_dev, cudaStream_t stream);
+
+/* One 128x128 tile of O = P . V (fp32) through the same TMEM-resident P
+ * (bf16) and tcgen05 BF16 MMA path as fp4attn_forward.  p_bf16_dev [128,128]
+ * (rows = queries, columns = keys), v_bf16_dev [128,128] (rows = keys),
+ * o_out_dev fp32 [128,128]. */
+int fp4attn_probe_pv_tile(const void* p_bf16_dev, const void* v_bf16_dev, float* o_out_dev,
+                          cudaStream_t stream);
+
+/* Runs the bounded mbarrier wait of the attention kernel on a barrier that
+ * nothing arrives at, with the given limit; the kernel must give up and write
+ * FP4ATTN_ERR_TIMEOUT into *status_dev (device int32, set to 0 first). */
+int fp4attn_probe_wait_timeout(int* status_dev, uint64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4ATTN_H */

@@ -1,0 +1,60 @@
+// Test-side kernels: NVFP4 -> fp32 dequantisation and element-wise fp32 ->
+// E2M1 / E4M3 conversion with the same device conversions the quantiser uses.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace fp4attn {
+
+namespace {
+
+// One thread per 16-value block: value = fl(fl(g * scale) * e2m1).
+__global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                               const float* g_ptr, int64_t nblocks, float* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nblocks) return;
+    const float g = g_ptr ? *g_ptr : 1.0f;
+    const float gs = __fmul_rn(g, ue4m3_value(scales[i]));
+    const uint2 c = *reinterpret_cast<const uint2*>(codes + i * 8);
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const uint32_t w = (e < 8) ? c.x : c.y;
+        v[e] = __fmul_rn(gs, e2m1_value((w >> (4 * (e & 7))) & 0xF));
+    }
+    float4* dst = reinterpret_cast<float4*>(out + i * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__global__ void encode_kernel(const float* __restrict__ x, int64_t n, uint8_t* e2m1, uint8_t* e4m3) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = x[i];
+        if (e2m1) e2m1[i] = (uint8_t)cvt_e2m1(v);
+        if (e4m3) e4m3[i] = (uint8_t)cvt_e4m3(v);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+                           float* out, cudaStream_t stream) {
+    const int64_t nblocks = rows * 8;
+    if (nblocks == 0) return cudaSuccess;
+    const int threads = 256;
+    dequant_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, stream>>>(
+        codes, scales, g, nblocks, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_encode_f32(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                              cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t want = (n + threads - 1) / threads;
+    const unsigned blocks = (unsigned)(want < 148 * 64 ? want : 148 * 64);
+    encode_kernel<<<blocks, threads, 0, stream>>>(x, n, e2m1, e4m3);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4attn

@@ -1,0 +1,75 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime_api.h>
+
+namespace fp4attn {
+
+constexpr int D = 128;
+
+// Workspace layout: [0,256) status word and spare; [256, 256 + 8*BH*128)
+// int64 key column sums; then one uint32 per head (ready counters).
+constexpr size_t WS_STATUS_BYTES = 256;
+inline size_t ws_ksum_offset() { return WS_STATUS_BYTES; }
+inline size_t ws_counter_offset(int64_t BH) { return WS_STATUS_BYTES + (size_t)BH * D * 8; }
+inline size_t ws_bytes(int64_t BH) {
+    size_t b = ws_counter_offset(BH) + (size_t)BH * 4;
+    return (b + 255) / 256 * 256;
+}
+
+struct QuantArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    int BH, N;
+    const float* gq;  // device scalar or nullptr (1.0)
+    const float* gk;
+    uint32_t flags;
+    uint8_t* q_codes;
+    uint8_t* q_scales;
+    uint8_t* k_codes;
+    uint8_t* k_scales;
+    float* k_mean;  // may be nullptr
+    long long* ksum;
+    unsigned* counters;
+    int* status;
+};
+
+cudaError_t launch_quantize_qk(const QuantArgs& a, cudaStream_t stream);
+
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+                           float* out, cudaStream_t stream);
+cudaError_t launch_encode_f32(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                              cudaStream_t stream);
+
+// Tensor-map encoder (driver entry point cuTensorMapEncodeTiled, looked up at
+// run time so the library needs no link to libcuda).
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle);
+
+struct FwdArgs {
+    const uint8_t* q_codes;
+    const uint8_t* q_scales;
+    const uint8_t* k_codes;
+    const uint8_t* k_scales;
+    const float* gq;
+    const float* gk;
+    const __nv_bfloat16* v;
+    int BH, N;
+    float softmax_scale;
+    __nv_bfloat16* o;
+    float* lse;
+    int* status;
+};
+
+// Returns 0 on success, else an fp4attn_status code.
+int launch_forward(const FwdArgs& a, cudaStream_t stream);
+int launch_probe_qk(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
+                    float* s_out, cudaStream_t stream);
+int launch_probe_pv(const __nv_bfloat16* p, const __nv_bfloat16* v, float* o_out,
+                    cudaStream_t stream);
+int launch_probe_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t stream);
+
+}  // namespace fp4attn

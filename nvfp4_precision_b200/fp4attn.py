@@ -1,0 +1,204 @@
+"""Python binding of the CUDA library's C ABI (include/fp4attn.h).
+
+Argument marshalling only: every step of the path runs in the library's
+kernels.  torch supplies device memory and the current stream.  Importing
+this module loads ``libfp4attn.so`` and raises if it is missing -- there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp4attn.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_CUDA = 3
+ERR_RANGE = 4
+ERR_TIMEOUT = 5
+ERR_WORKSPACE = 6
+NO_SMOOTH_K = 1
+NO_HADAMARD = 2
+
+EXPORTS = (
+    "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_forward", "fp4attn_dequant",
+    "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
+    "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
+)
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("D", ctypes.c_int32)]
+
+
+class Fp4AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library {LIB_PATH} is missing; build it with "
+                          f"`python -m nvfp4_precision_b200.build` (there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, U32, U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
+    L.fp4attn_workspace_bytes.restype = ctypes.c_size_t
+    L.fp4attn_workspace_bytes.argtypes = [Shape]
+    L.fp4attn_quantize_qk.restype = ctypes.c_int
+    L.fp4attn_quantize_qk.argtypes = [P, P, Shape, P, P, U32, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_forward.restype = ctypes.c_int
+    L.fp4attn_forward.argtypes = [P, P, P, P, P, P, P, Shape, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_dequant.restype = ctypes.c_int
+    L.fp4attn_dequant.argtypes = [P, P, P, Shape, P, P]
+    L.fp4attn_read_status.restype = ctypes.c_int
+    L.fp4attn_read_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int)]
+    L.fp4attn_reset_status.restype = ctypes.c_int
+    L.fp4attn_reset_status.argtypes = [P, P]
+    L.fp4attn_status_string.restype = ctypes.c_char_p
+    L.fp4attn_status_string.argtypes = [ctypes.c_int]
+    L.fp4attn_encode_f32.restype = ctypes.c_int
+    L.fp4attn_encode_f32.argtypes = [P, I64, P, P, P]
+    L.fp4attn_probe_qk_tile.restype = ctypes.c_int
+    L.fp4attn_probe_qk_tile.argtypes = [P, P, P, P, P, P]
+    L.fp4attn_probe_pv_tile.restype = ctypes.c_int
+    L.fp4attn_probe_pv_tile.argtypes = [P, P, P, P]
+    L.fp4attn_probe_wait_timeout.restype = ctypes.c_int
+    L.fp4attn_probe_wait_timeout.argtypes = [P, U64, P]
+    return L
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.fp4attn_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise Fp4AttnError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def shape_of(t: torch.Tensor) -> Shape:
+    B, H, N, D = t.shape
+    return Shape(B, H, N, D)
+
+
+def fp4attn_workspace_bytes(B: int, H: int, N: int, D: int = 128) -> int:
+    return int(lib.fp4attn_workspace_bytes(Shape(B, H, N, D)))
+
+
+def new_workspace(B: int, H: int, N: int, device="cuda") -> torch.Tensor:
+    n = fp4attn_workspace_bytes(B, H, N)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def fp4attn_quantize_qk(q: torch.Tensor, k: torch.Tensor, q_gscale: Optional[torch.Tensor] = None,
+                        k_gscale: Optional[torch.Tensor] = None, flags: int = 0, out: Optional[dict] = None,
+                        k_mean: bool = True, workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Smooth K + Hadamard + NVFP4 pack of bf16 [B,H,N,128] Q and K.
+
+    Returns dict(q_codes, q_scales, k_codes, k_scales, k_mean, workspace)."""
+    assert q.dtype == torch.bfloat16 and k.dtype == torch.bfloat16 and q.shape == k.shape
+    assert q.is_contiguous() and k.is_contiguous()
+    B, H, N, D = q.shape
+    dev = q.device
+    if out is None:
+        out = dict(q_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
+                   q_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
+                   k_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
+                   k_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
+                   k_mean=torch.empty((B, H, 128), dtype=torch.float32, device=dev) if k_mean else None)
+    if workspace is None:
+        workspace = new_workspace(B, H, N, dev)
+    rc = lib.fp4attn_quantize_qk(_ptr(q), _ptr(k), Shape(B, H, N, D), _ptr(q_gscale), _ptr(k_gscale),
+                                 int(flags), _ptr(out["q_codes"]), _ptr(out["q_scales"]), _ptr(out["k_codes"]),
+                                 _ptr(out["k_scales"]), _ptr(out.get("k_mean")), _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_quantize_qk")
+    out["workspace"] = workspace
+    return out
+
+
+def fp4attn_forward(q_codes, q_scales, k_codes, k_scales, v: torch.Tensor, q_gscale=None, k_gscale=None,
+                    softmax_scale: float = 0.0, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Non-causal attention over NVFP4 Q/K and bf16 V.  Returns (O, lse or None)."""
+    assert v.dtype == torch.bfloat16 and v.is_contiguous()
+    B, H, N, D = v.shape
+    if o is None:
+        o = torch.empty_like(v)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
+    if workspace is None:
+        workspace = new_workspace(B, H, N, v.device)
+        workspace.zero_()
+    rc = lib.fp4attn_forward(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(q_gscale),
+                             _ptr(k_gscale), _ptr(v), Shape(B, H, N, D), float(softmax_scale), _ptr(o), _ptr(lse),
+                             _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_forward")
+    return o, lse
+
+
+def fp4attn_dequant(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    B, H, N, _ = codes.shape
+    out = torch.empty((B, H, N, 128), dtype=torch.float32, device=codes.device)
+    rc = lib.fp4attn_dequant(_ptr(codes), _ptr(scales), _ptr(gscale), Shape(B, H, N, 128), _ptr(out),
+                             _stream(stream))
+    _check(rc, "fp4attn_dequant")
+    return out
+
+
+def fp4attn_read_status(workspace: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int(-1)
+    _check(lib.fp4attn_read_status(_ptr(workspace), _stream(stream), ctypes.byref(v)), "fp4attn_read_status")
+    return v.value
+
+
+def fp4attn_reset_status(workspace: torch.Tensor, stream=None):
+    _check(lib.fp4attn_reset_status(_ptr(workspace), _stream(stream)), "fp4attn_reset_status")
+
+
+def fp4attn_encode_f32(x: torch.Tensor, stream=None):
+    assert x.dtype == torch.float32 and x.is_contiguous()
+    e2m1 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    e4m3 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib.fp4attn_encode_f32(_ptr(x), x.numel(), _ptr(e2m1), _ptr(e4m3), _stream(stream)), "fp4attn_encode_f32")
+    return e2m1, e4m3
+
+
+def fp4attn_probe_qk_tile(q_codes, q_scales, k_codes, k_scales, stream=None) -> torch.Tensor:
+    s = torch.empty((128, 128), dtype=torch.float32, device=q_codes.device)
+    _check(lib.fp4attn_probe_qk_tile(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(s),
+                                     _stream(stream)), "fp4attn_probe_qk_tile")
+    return s
+
+
+def fp4attn_probe_pv_tile(p: torch.Tensor, v: torch.Tensor, stream=None) -> torch.Tensor:
+    o = torch.empty((128, 128), dtype=torch.float32, device=p.device)
+    _check(lib.fp4attn_probe_pv_tile(_ptr(p), _ptr(v), _ptr(o), _stream(stream)), "fp4attn_probe_pv_tile")
+    return o
+
+
+def fp4attn_probe_wait_timeout(limit_ns: int, stream=None) -> int:
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib.fp4attn_probe_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)), "fp4attn_probe_wait_timeout")
+    return int(status.item())

@@ -100,11 +100,13 @@ def _draw_head(child: np.random.SeedSequence, w: Workload, tail: bool) -> np.nda
     return x
 
 
-def generate(w: Workload, tensors=("q", "k", "v")) -> dict:
+def generate(w: Workload, tensors=("q", "k", "v"), heads=None) -> dict:
     """Return CPU bf16 tensors ``[B, H, N, 128]`` for the requested names.
 
     The draw for every (tensor, head) comes from its own child stream, so a
-    tensor's values do not depend on which other tensors were requested.
+    tensor's values do not depend on which other tensors or heads were
+    requested.  ``heads`` (flat b*H + h indices) restricts the draw to those
+    heads; the result then has shape ``[1, len(heads), N, 128]``.
     """
     BH = w.B * w.H
     root = np.random.SeedSequence(w.seed)
@@ -117,25 +119,27 @@ def generate(w: Workload, tensors=("q", "k", "v")) -> dict:
     if w.n_outliers > 0:
         outl = np.sort(g0.choice(D, size=w.n_outliers, replace=False))
 
+    sel = list(range(BH)) if heads is None else [int(h) for h in heads]
     out = {}
     index = {"q": 0, "k": 1, "v": 2}
     for name in tensors:
         if name == "v" and not w.with_v:
             continue
         t = index[name]
-        res = torch.empty((BH, w.N, D), dtype=torch.bfloat16)
+        res = torch.empty((len(sel), w.N, D), dtype=torch.bfloat16)
 
-        def work(bh, t=t, name=name, res=res):
+        def work(i, t=t, name=name, res=res):
+            bh = sel[i]
             x = _draw_head(children[1 + t * BH + bh], w, tail=True)
             if outl is not None and name in ("q", "k"):
                 x[:, outl] *= np.float32(w.outlier_factor)
             if offset is not None and name == "k":
                 x += offset[bh][None, :]
-            res[bh] = torch.from_numpy(x).to(torch.bfloat16)
+            res[i] = torch.from_numpy(x).to(torch.bfloat16)
 
         with ThreadPoolExecutor(_threads()) as ex:
-            list(ex.map(work, range(BH)))
-        out[name] = res.view(w.B, w.H, w.N, D)
+            list(ex.map(work, range(len(sel))))
+        out[name] = res.view(w.B, w.H, w.N, D) if heads is None else res.view(1, len(sel), w.N, D)
     out["outlier_channels"] = outl
     return out
 

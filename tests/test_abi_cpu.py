@@ -1,0 +1,81 @@
+"""The C-ABI library loads and exports every symbol include/fp4attn.h declares,
+and argument validation rejects bad calls before anything is launched.
+CPU only: no call here reaches the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from nvfp4_precision_b200 import build
+    build.build()
+    from nvfp4_precision_b200 import fp4attn
+    return fp4attn
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(fp4attn_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported(fa):
+    names = declared_functions()
+    assert {"fp4attn_quantize_qk", "fp4attn_forward", "fp4attn_dequant"} <= names
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+    assert set(fa.EXPORTS) >= names
+
+
+def test_status_strings_and_workspace(fa):
+    assert fa.status_string(0) == "ok"
+    assert "wait" in fa.status_string(fa.ERR_TIMEOUT)
+    assert fa.status_string(99) == "unknown status"
+    ws = fa.fp4attn_workspace_bytes(1, 48, 109568)
+    assert ws >= 48 * 128 * 8 + 4 and ws % 256 == 0
+    assert fa.fp4attn_workspace_bytes(0, 0, 0) > 0
+
+
+def _q(fa, shape, ws=ctypes.c_void_p(256), wsb=1 << 20, flags=0, ptr=ctypes.c_void_p(4096)):
+    return fa.lib.fp4attn_quantize_qk(ptr, ptr, shape, None, None, flags, ptr, ptr, ptr, ptr, None, ws, wsb, None)
+
+
+def test_quantize_validation_before_launch(fa):
+    S = fa.Shape
+    assert _q(fa, S(1, 1, 128, 64)) == fa.ERR_UNSUPPORTED          # D != 128
+    assert _q(fa, S(1, -1, 128, 128)) == fa.ERR_INVALID_ARG        # negative size
+    assert _q(fa, S(1, 1, 1 << 19, 128)) == fa.ERR_UNSUPPORTED     # N beyond the exact-sum range
+    assert _q(fa, S(1, 1, 128, 128), flags=8) == fa.ERR_INVALID_ARG
+    assert _q(fa, S(1, 1, 128, 128), ws=None) == fa.ERR_WORKSPACE
+    assert _q(fa, S(1, 1, 128, 128), wsb=16) == fa.ERR_WORKSPACE
+    assert _q(fa, S(1, 1, 128, 128), ws=ctypes.c_void_p(258)) == fa.ERR_WORKSPACE
+    assert _q(fa, S(1, 1, 128, 128), ptr=ctypes.c_void_p(4100)) == fa.ERR_INVALID_ARG  # misaligned
+
+
+def test_forward_validation_before_launch(fa):
+    S = fa.Shape
+    p = ctypes.c_void_p(4096)
+    f = fa.lib.fp4attn_forward
+    assert f(p, p, p, p, None, None, p, S(1, 1, 128, 96), 0.0, p, None, p, 1 << 20, None) == fa.ERR_UNSUPPORTED
+    assert f(p, p, p, p, None, None, p, S(1, 1, 128, 128), 0.0, p, None, None, 0, None) == fa.ERR_WORKSPACE
+    assert f(None, p, p, p, None, None, p, S(1, 1, 128, 128), 0.0, p, None, p, 1 << 20, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, p, p, None, None, p, S(1, 1, 128, 128), float("nan"), p, None, p, 1 << 20, None) \
+        == fa.ERR_INVALID_ARG
+    assert f(p, p, p, p, None, None, p, S(1, 1, 128, 128), 0.0, p, ctypes.c_void_p(4098), p, 1 << 20, None) \
+        == fa.ERR_INVALID_ARG
+
+
+def test_probe_validation(fa):
+    assert fa.lib.fp4attn_probe_qk_tile(None, None, None, None, None, None) == fa.ERR_INVALID_ARG
+    assert fa.lib.fp4attn_probe_wait_timeout(None, 1000, None) == fa.ERR_INVALID_ARG
+    assert fa.lib.fp4attn_encode_f32(None, 5, None, None, None) == fa.ERR_INVALID_ARG

@@ -1,0 +1,130 @@
+"""GPU parity of the quantisation prologue (smooth K + Hadamard + NVFP4 pack)
+and of the device codecs, bit-exact against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_precision_b200 import synth
+
+from gpu_helpers import fa, gpu_prologue, oracle_prologue
+
+pytestmark = pytest.mark.gpu
+
+KEYS = ("q_codes", "q_scales", "k_codes", "k_scales", "k_mean")
+
+
+def assert_prologue_equal(g, o, what):
+    assert g["status"] == 0, f"{what}: device status {g['status']}"
+    for key in KEYS:
+        if not np.array_equal(g[key], o[key]):
+            bad = np.argwhere(g[key] != o[key])
+            raise AssertionError(f"{what}: {key} differs at {bad.shape[0]} places, first {bad[:3].tolist()}")
+
+
+def _fp32_range(lo_exp, hi_exp, step=1):
+    lo = np.float32(2.0 ** lo_exp).view(np.uint32)
+    hi = np.float32(2.0 ** hi_exp).view(np.uint32)
+    return np.arange(lo, hi, step, dtype=np.uint32).view(np.float32)
+
+
+def test_device_codecs_match_oracle_over_dense_fp32_sweep():
+    # every fp32 value with magnitude in [2^-12, 2^10) (both signs), plus zeros,
+    # tiny, huge and infinite values
+    pos = _fp32_range(-12, 10)
+    extra = np.array([0.0, 1e-30, 2.0 ** -126, 2.0 ** -149, 3e38, np.inf], np.float32)
+    chunks = [pos, -pos, extra, -extra]
+    for x in chunks:
+        xt = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        e2m1, e4m3 = fa().fp4attn_encode_f32(xt)
+        e2m1 = e2m1.cpu().numpy()
+        want = oracle.e2m1_encode(x)
+        bad = np.nonzero(e2m1 != want)[0]
+        assert bad.size == 0, [(float(x[i]), int(e2m1[i]), int(want[i])) for i in bad[:8]]
+        # the quantiser only converts t = amax/6/g >= +0, so compare non-negative inputs
+        # (negative zero keeps its sign bit in E4M3)
+        nonneg = (x >= 0) & ~np.signbit(x)
+        e4 = e4m3.cpu().numpy()[nonneg]
+        want4 = oracle.ue4m3_encode(x[nonneg])
+        bad = np.nonzero(e4 != want4)[0]
+        assert bad.size == 0, [(float(x[nonneg][i]), int(e4[i]), int(want4[i])) for i in bad[:8]]
+
+
+@pytest.mark.parametrize("name,B,H,N,extra", [
+    ("one_row", 1, 1, 1, {}),
+    ("ragged127", 1, 3, 127, dict(k_offset_std=2.0)),
+    ("ragged1000", 2, 2, 1000, dict(k_offset_std=2.0, n_outliers=2, outlier_factor=20.0)),
+    ("heavy_tail", 1, 4, 4096, dict(dist="student_t3", n_outliers=4, outlier_factor=50.0)),
+])
+def test_prologue_bit_exact_small(name, B, H, N, extra):
+    d = synth.generate(synth.custom(name, B, H, N, seed=100 + N, **extra), ("q", "k"))
+    assert_prologue_equal(gpu_prologue(d), oracle_prologue(d), name)
+
+
+@pytest.mark.parametrize("flags", [0, 1, 2, 3])
+def test_prologue_bit_exact_tiny_all_flags(flags):
+    d = synth.generate(synth.WORKLOADS["tiny"], ("q", "k"))
+    assert_prologue_equal(gpu_prologue(d, flags=flags), oracle_prologue(d, flags=flags), f"tiny flags={flags}")
+
+
+def test_prologue_bit_exact_global_scales():
+    d = synth.generate(synth.WORKLOADS["tiny"], ("q", "k"))
+    g = gpu_prologue(d, gq=0.37, gk=3.1)
+    o = oracle_prologue(d, gq=np.float32(0.37), gk=np.float32(3.1))
+    assert_prologue_equal(g, o, "tiny g!=1")
+
+
+def test_prologue_bit_exact_mid():
+    d = synth.generate(synth.WORKLOADS["mid"], ("q", "k"))
+    assert_prologue_equal(gpu_prologue(d), oracle_prologue(d), "mid")
+
+
+def test_prologue_key_permutation_gives_permuted_codes():
+    """The key mean is an exact integer sum: permuting keys permutes the codes."""
+    d = synth.generate(synth.custom("perm", 1, 2, 3000, seed=9, k_offset_std=2.0), ("q", "k"))
+    g1 = gpu_prologue(d)
+    perm = torch.from_numpy(np.random.default_rng(0).permutation(3000))
+    d2 = dict(q=d["q"], k=d["k"][:, :, perm].contiguous())
+    g2 = gpu_prologue(d2)
+    assert np.array_equal(g2["k_mean"], g1["k_mean"])
+    assert np.array_equal(g2["k_codes"], g1["k_codes"][:, :, perm.numpy()])
+    assert np.array_equal(g2["k_scales"], g1["k_scales"][:, :, perm.numpy()])
+
+
+@pytest.mark.parametrize("name", ["clip5s", "prologue_stress"])
+def test_prologue_bit_exact_full_size(name):
+    d = synth.generate(synth.WORKLOADS[name], ("q", "k"))
+    assert_prologue_equal(gpu_prologue(d), oracle_prologue(d), name)
+
+
+def test_dequant_matches_oracle():
+    d = synth.generate(synth.WORKLOADS["tiny"], ("q", "k"))
+    o = oracle_prologue(d)
+    codes = torch.from_numpy(o["k_codes"]).cuda()
+    scales = torch.from_numpy(o["k_scales"]).cuda()
+    for g in (None, 0.75):
+        gt = None if g is None else torch.tensor([g], dtype=torch.float32, device="cuda")
+        got = fa().fp4attn_dequant(codes, scales, gt).cpu().numpy()
+        want = oracle.dequant(o["k_codes"], o["k_scales"], 1.0 if g is None else g)
+        assert np.array_equal(got, want)
+
+
+def test_range_errors_are_reported():
+    d = synth.generate(synth.custom("bad", 1, 1, 256, seed=3), ("q", "k"))
+    k = d["k"].clone()
+    k[0, 0, 5, 7] = 2.0 ** 21
+    assert gpu_prologue(dict(q=d["q"], k=k))["status"] == fa().ERR_RANGE
+    q = d["q"].clone()
+    q[0, 0, 9, 1] = float("nan")
+    assert gpu_prologue(dict(q=q, k=d["k"]))["status"] == fa().ERR_RANGE
+    assert gpu_prologue(d, gq=-1.0)["status"] == fa().ERR_RANGE
+    assert gpu_prologue(d)["status"] == 0
+
+
+def test_empty_shapes_are_no_ops():
+    q = torch.zeros((1, 0, 128, 128), dtype=torch.bfloat16, device="cuda")
+    out = fa().fp4attn_quantize_qk(q, q)
+    assert fa().fp4attn_read_status(out["workspace"]) == 0
+    q = torch.zeros((2, 3, 0, 128), dtype=torch.bfloat16, device="cuda")
+    out = fa().fp4attn_quantize_qk(q, q)
+    assert out["q_codes"].numel() == 0
