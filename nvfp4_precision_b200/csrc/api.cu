@@ -127,6 +127,7 @@ int fp4attn_quantize_qk(const void* q, const void* k, fp4attn_shape s, const flo
     a.k_mean = k_mean;
     a.ksum = reinterpret_cast<long long*>(ws + ws_ksum_offset());
     a.counters = reinterpret_cast<unsigned*>(ws + ws_counter_offset(heads(s)));
+    a.ticket = reinterpret_cast<unsigned*>(ws + WS_TICKET_OFFSET);
     a.status = reinterpret_cast<int*>(ws);
     return launch_status(launch_quantize_qk(a, stream));
 }

@@ -4,12 +4,15 @@
 // Method: FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention":
 // queries and keys are quantised for an NVFP4 attention kernel; P and V stay
 // in BF16.  This kernel is written for sm_100a:
-//   * one CTA per (head, 128-query tile); 192 threads in three roles
-//       warps 0-3  softmax, O correction and epilogue; thread i owns query
-//                  row i, which is TMEM lane i;
-//       warp 4     TMA producer: Q tile once, then K codes, K scales and V
-//                  tiles of 128 keys into a STAGES-deep shared-memory ring;
-//       warp 5     TMEM owner and MMA issuer: stages the scale factors into
+//   * one CTA per (head, 128-query tile); 320 threads in three roles
+//       warps 0-7  softmax, O correction and epilogue; query row r is TMEM
+//                  lane r and is shared by warps r/32 (keys 0-63 of each
+//                  tile) and r/32 + 4 (keys 64-127), which exchange their
+//                  partial row maxima through shared memory every tile;
+//       warp 8     producer: scale-factor atoms (plain loads) and TMA copies
+//                  of Q once, then K codes and V tiles of 128 keys into a
+//                  STAGES-deep shared-memory ring;
+//       warp 9     TMEM owner and MMA issuer: stages the scale factors into
 //                  TMEM (tcgen05.cp) and issues S = Q K^T with
 //                  tcgen05.mma kind::mxf4nvf4 (block16 scales) and
 //                  O += P V with tcgen05.mma kind::f16 (P read from TMEM);
@@ -18,7 +21,9 @@
 //     written as bf16 pairs over the first 64 columns of its S buffer;
 //   * online softmax in the log2 domain with a lazy rescale: the running max
 //     only moves when a tile's max exceeds it by more than 8 (so p <= 256),
-//     and O is rescaled in TMEM only then.
+//     and O is rescaled in TMEM only then; exponentials are split between
+//     the MUFU unit and a polynomial on the FMA pipe, with packed fp32x2
+//     arithmetic for the scale, the polynomial and the row sums.
 // Every wait is bounded; a wait that runs out raises FP4ATTN_ERR_TIMEOUT in
 // the status word and the CTA winds down (waiting for its own copies and MMAs)
 // instead of hanging.
@@ -34,9 +39,13 @@ namespace {
 constexpr int BM = 128;  // query rows per CTA
 constexpr int BN = 128;  // keys per tile
 constexpr int STAGES = 3;
-constexpr int FWD_THREADS = 192;
-constexpr int WARP_PRODUCER = 4;
-constexpr int WARP_MMA = 5;
+constexpr int SOFTMAX_WARPS = 8;
+constexpr int FWD_THREADS = 32 * (SOFTMAX_WARPS + 2);
+constexpr int WARP_PRODUCER = SOFTMAX_WARPS;
+constexpr int WARP_MMA = SOFTMAX_WARPS + 1;
+// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
+// and the rest to MUFU ex2 (MUFU issues 16 per clock per SM).
+constexpr int POLY_PAIRS_PER_8 = 3;
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0;
@@ -45,7 +54,6 @@ constexpr uint32_t TM_SFQ = 384;
 constexpr uint32_t TM_SFK = 392;
 
 constexpr uint32_t CODE_TILE_BYTES = 128 * 64;    // 128 rows x 128 E2M1 values
-constexpr uint32_t SCALE_TILE_BYTES = 128 * 8;    // 128 rows x 8 UE4M3 scales
 constexpr uint32_t V_PANEL_BYTES = 128 * 64 * 2;  // 128 keys x 64 channels bf16
 constexpr uint32_t V_TILE_BYTES = 2 * V_PANEL_BYTES;
 
@@ -62,9 +70,7 @@ struct __align__(1024) FwdSmem {
     uint8_t v[STAGES][V_TILE_BYTES];      // two 64-channel panels, 128B swizzle
     uint8_t kc[STAGES][CODE_TILE_BYTES];  // 64B swizzle
     uint8_t qc[CODE_TILE_BYTES];          // 64B swizzle
-    uint64_t ks_raw[STAGES][128];         // row-major scales, one uint64 per key
-    uint64_t qs_raw[128];
-    uint8_t ks_atom[2][2][512];           // scale-factor atoms for tcgen05.cp
+    uint8_t ks_atom[STAGES][2][512];      // scale-factor atoms for tcgen05.cp
     uint8_t qs_atom[2][512];
     uint64_t bar_q_full;
     uint64_t bar_kv_full[STAGES];
@@ -73,11 +79,16 @@ struct __align__(1024) FwdSmem {
     uint64_t bar_p_ready;
     uint64_t bar_o_done;
     uint64_t bar_final;
+    uint64_t bar_pair[4][2];      // per row quarter, per tile parity: both halves' maxima are in
+    float red_max[2][2][128];     // [tile parity][half][row] partial row maxima
+    float red_sum[2][128];        // [half][row] partial row sums, at the end
     uint32_t tmem_base;
     int abort_flag;
 };
 
 struct FwdParams {
+    const uint64_t* q_scales;  // one uint64 (8 UE4M3 bytes) per row
+    const uint64_t* k_scales;
     int N;
     int n_kt;
     float scale_log2;  // softmax_scale * log2(e)
@@ -110,17 +121,20 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
     return mbar_wait(bar, parity, &dummy_abort, nullptr, kDrainLimitNs);
 }
 
-// Row-major scales (one uint64 = 8 UE4M3 bytes per row) -> two 512-byte
-// atoms (channels 0-63 and 64-127).  Atom line r (16 bytes) holds, for rows
-// r, r+32, r+64, r+96, the four scales of that 64-channel chunk; tcgen05.cp
-// 32x128b.warpx4 then puts line r in TMEM lane r of every sub-partition.
-// Executed by one full warp (lane = line).
-__device__ __forceinline__ void stage_scale_atoms(const uint64_t* raw, uint8_t* atom0, uint8_t* atom1,
-                                                  int lane) {
+// Scales of 128 rows (row-major, one uint64 = 8 UE4M3 bytes per row) -> two
+// 512-byte atoms (channels 0-63 and 64-127).  Atom line r (16 bytes) holds,
+// for rows r, r+32, r+64, r+96, the four scales of that 64-channel chunk;
+// tcgen05.cp 32x128b.warpx4 then puts line r in TMEM lane r of every
+// sub-partition.  One full warp, lane = line; rows at or beyond n_rows read
+// as zero.  Plain 8-byte loads: a row's scales start at any multiple of 8
+// bytes, which a bulk tensor copy could not address.
+__device__ __forceinline__ void load_scale_atoms(const uint64_t* rows, int n_rows, uint8_t* atom0,
+                                                 uint8_t* atom1, int lane) {
     uint32_t lo[4], hi[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const uint64_t w = raw[lane + 32 * c];
+        const int r = lane + 32 * c;
+        const uint64_t w = (r < n_rows) ? __ldg(reinterpret_cast<const unsigned long long*>(rows) + r) : 0ull;
         lo[c] = (uint32_t)w;
         hi[c] = (uint32_t)(w >> 32);
     }
@@ -167,8 +181,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t p_col, const ui
 }
 
 __global__ void __launch_bounds__(FWD_THREADS, 1)
-    fwd_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_qs,
-               const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_ks,
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_kc,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem& sm = *align1024<FwdSmem>(smem_raw);
@@ -187,9 +200,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
         mbar_init(smem_u32(&sm.bar_s_full[0]), 1);
         mbar_init(smem_u32(&sm.bar_s_full[1]), 1);
-        mbar_init(smem_u32(&sm.bar_p_ready), 4 * 32);
+        mbar_init(smem_u32(&sm.bar_p_ready), SOFTMAX_WARPS * 32);
         mbar_init(smem_u32(&sm.bar_o_done), 1);
         mbar_init(smem_u32(&sm.bar_final), 1);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(smem_u32(&sm.bar_pair[q][0]), 64);
+            mbar_init(smem_u32(&sm.bar_pair[q][1]), 64);
+        }
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -199,9 +216,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     }
     if (warp == WARP_PRODUCER && lane == 0) {
         prefetch_tmap(&tm_qc);
-        prefetch_tmap(&tm_qs);
         prefetch_tmap(&tm_kc);
-        prefetch_tmap(&tm_ks);
         prefetch_tmap(&tm_v);
     }
     tc_fence_before();
@@ -213,42 +228,50 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 
     if (warp == WARP_PRODUCER) {
         // ------------------------------------------------------ producer --
+        // All 32 lanes stage the scale atoms; lane 0 arms the barrier and
+        // issues the bulk tensor copies after the atoms are written.
+        const uint64_t* qs_head = p.q_scales + (size_t)bh * N;
+        const uint64_t* ks_head = p.k_scales + (size_t)bh * N;
+        const uint32_t qf = smem_u32(&sm.bar_q_full);
+        load_scale_atoms(qs_head + q0, N - q0, sm.qs_atom[0], sm.qs_atom[1], lane);
+        fence_proxy_async_smem();
+        __syncwarp();
         if (lane == 0) {
-            const uint32_t qf = smem_u32(&sm.bar_q_full);
-            mbar_arrive_expect_tx(qf, CODE_TILE_BYTES + SCALE_TILE_BYTES);
+            mbar_arrive_expect_tx(qf, CODE_TILE_BYTES);
             tma_load_3d(smem_u32(sm.qc), &tm_qc, 0, q0, bh, qf);
-            tma_load_1d(smem_u32(sm.qs_raw), &tm_qs, bh * N + q0, qf);
-            int issued = 0;
-            for (int j = 0; j < T; ++j) {
-                const int s = j % STAGES;
-                if (j >= STAGES) {
-                    if (!mbar_wait(smem_u32(&sm.bar_kv_empty[s]), ((j / STAGES) - 1) & 1, abort_flag,
-                                   p.status, limit))
-                        break;
-                }
+        }
+        int issued = 0;
+        for (int j = 0; j < T; ++j) {
+            const int s = j % STAGES;
+            if (j >= STAGES) {
+                if (!warp_wait(smem_u32(&sm.bar_kv_empty[s]), ((j / STAGES) - 1) & 1, abort_flag, p.status,
+                               limit))
+                    break;
+            }
+            const int k0 = j * BN;
+            load_scale_atoms(ks_head + k0, N - k0, sm.ks_atom[s][0], sm.ks_atom[s][1], lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
                 const uint32_t full = smem_u32(&sm.bar_kv_full[s]);
-                mbar_arrive_expect_tx(full, CODE_TILE_BYTES + SCALE_TILE_BYTES + V_TILE_BYTES);
-                const int k0 = j * BN;
+                mbar_arrive_expect_tx(full, CODE_TILE_BYTES + V_TILE_BYTES);
                 tma_load_3d(smem_u32(sm.kc[s]), &tm_kc, 0, k0, bh, full);
-                tma_load_1d(smem_u32(sm.ks_raw[s]), &tm_ks, bh * N + k0, full);
                 tma_load_3d(smem_u32(sm.v[s]), &tm_v, 0, k0, bh, full);
                 tma_load_3d(smem_u32(sm.v[s]) + V_PANEL_BYTES, &tm_v, 64, k0, bh, full);
-                issued = j + 1;
             }
-            if (*abort_flag) {
-                // wind down: let this CTA's own copies land before it exits
-                drain_wait(qf, 0);
-                for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-                    drain_wait(smem_u32(&sm.bar_kv_full[i % STAGES]), (i / STAGES) & 1);
-            }
+            __syncwarp();
+            issued = j + 1;
+        }
+        if (lane == 0 && *abort_flag) {
+            // wind down: let this CTA's own copies land before it exits
+            drain_wait(qf, 0);
+            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+                drain_wait(smem_u32(&sm.bar_kv_full[i % STAGES]), (i / STAGES) & 1);
         }
     } else if (warp == WARP_MMA) {
         // ----------------------------------------------------------- MMA --
         bool ok = warp_wait(smem_u32(&sm.bar_q_full), 0, abort_flag, p.status, limit);
         if (ok) {
-            stage_scale_atoms(sm.qs_raw, sm.qs_atom[0], sm.qs_atom[1], lane);
-            fence_proxy_async_smem();
-            __syncwarp();
             if (lane == 0) {
                 tc_fence_after();
                 tmem_cp_32x128b_x4(tmem + TM_SFQ, atom_desc(sm.qs_atom[0]));
@@ -274,14 +297,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 ok = false;
                 break;
             }
-            stage_scale_atoms(sm.ks_raw[s], sm.ks_atom[b][0], sm.ks_atom[b][1], lane);
-            fence_proxy_async_smem();
-            __syncwarp();
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t sfk = TM_SFK + 8u * b;
-                tmem_cp_32x128b_x4(tmem + sfk, atom_desc(sm.ks_atom[b][0]));
-                tmem_cp_32x128b_x4(tmem + sfk + 4, atom_desc(sm.ks_atom[b][1]));
+                tmem_cp_32x128b_x4(tmem + sfk, atom_desc(sm.ks_atom[s][0]));
+                tmem_cp_32x128b_x4(tmem + sfk + 4, atom_desc(sm.ks_atom[s][1]));
                 issue_qk(tmem, TM_S0 + 128u * b, sm.qc, sm.kc[s], sfk);
                 tc_commit(smem_u32(&sm.bar_s_full[b]));
             }
@@ -300,8 +320,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ softmax warps --
-        const int row = 32 * warp + lane;
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const int quad = warp & 3;   // TMEM sub-partition: rows 32*quad ..
+        const int half = warp >> 2;  // keys 64*half .. 64*half+63 of each tile
+        const int row = 32 * quad + lane;
+        const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
         float gq = 1.0f, gk = 1.0f;
         if (p.gq) gq = *p.gq;
         if (p.gk) gk = *p.gk;
@@ -309,8 +331,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             if (threadIdx.x == 0) atomicCAS(p.status, 0, (int)FP4ATTN_ERR_RANGE);
         }
         const float c = p.scale_log2 * gq * gk;
+        const float2 c2 = make_float2(c, c);
         float m_run = -INFINITY;
-        float l = 0.0f;
+        float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
         bool ok = true;
         for (int j = 0; j < T; ++j) {
             const int b = j & 1;
@@ -320,47 +344,66 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld32(s_addr + 32u * q, sr[q]);
+            uint32_t sr[2][32];
+            tmem_ld32(s_addr + 64u * half, sr[0]);
+            tmem_ld32(s_addr + 64u * half + 32u, sr[1]);
             tmem_wait_ld();
-            const int nvalid = N - j * BN;
-            if (nvalid < BN) {
+            const int nvalid = N - j * BN - 64 * half;
+            if (nvalid < 64) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int q = 0; q < 2; ++q)
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (32 * q + i >= nvalid) sr[q][i] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            // partial row max of this half: a tree of three-input maxima
+            float a[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[q][i]));
-            const float mx_scaled = mx * c;
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t* v = &sr[k >> 2][(k & 3) * 8];
+                a[k] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                             fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                             fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+            }
+            const float pmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+            // exchange with the other half of the row (all S reads of the tile are done after this)
+            sm.red_max[b][half][row] = pmax;
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.bar_pair[quad][b]));
+            if (!warp_wait(smem_u32(&sm.bar_pair[quad][b]), (j >> 1) & 1, abort_flag, p.status, limit)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float mx = fmaxf(pmax, sm.red_max[b][half ^ 1][row]) * c;
             float alpha = 1.0f;
             bool rescale = false;
-            if (mx_scaled > m_run + 8.0f) {
-                alpha = ex2_approx(m_run - mx_scaled);
-                m_run = mx_scaled;
+            if (mx > m_run + 8.0f) {
+                alpha = ex2_approx(m_run - mx);
+                m_run = mx;
                 rescale = true;
+                const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) lacc[k] = __fmul2_rn(lacc[k], a2);
             }
-            const float neg_m = -m_run;
-            float rowsum = 0.0f;
-            uint32_t pk[2][32];
+            const float2 negm = make_float2(-m_run, -m_run);
+            uint32_t pk[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][i]), c, neg_m));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][i + 1]), c, neg_m));
-                    rowsum += p0 + p1;
-                    pk[q >> 1][(q & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
+            for (int k = 0; k < 32; ++k) {
+                const float2 s2 = make_float2(__uint_as_float(sr[k >> 4][(2 * k) & 31]),
+                                              __uint_as_float(sr[k >> 4][(2 * k + 1) & 31]));
+                const float2 x = __ffma2_rn(s2, c2, negm);
+                float2 pv;
+                if ((k & 7) < POLY_PAIRS_PER_8) {
+                    pv = exp2_poly2(x);
+                } else {
+                    pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                 }
+                lacc[k & 3] = __fadd2_rn(lacc[k & 3], pv);
+                pk[k] = pack_bf16x2(pv.x, pv.y);
             }
-            l = l * alpha + rowsum;
-            tmem_st32(s_addr, pk[0]);
-            tmem_st32(s_addr + 32u, pk[1]);
+            // P (bf16 pairs) over this half's 32 columns of the S buffer
+            tmem_st32(s_addr + 32u * half, pk);
             tmem_wait_st();
             if (j >= 1) {
                 // O holds the sum up to tile j-1 once that tile's P.V is done
@@ -368,16 +411,23 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     ok = false;
                     break;
                 }
-                if (rescale) {
+                // tcgen05.ld/st are warp-collective: the whole warp takes this
+                // branch when any of its rows needs it (alpha is 1 elsewhere)
+                if (__any_sync(0xffffffffu, rescale)) {
                     tc_fence_after();
-                    const uint32_t o_addr = tmem + lane_base + TM_O;
+                    const uint32_t o_addr = tmem + lane_base + TM_O + 64u * half;
+                    const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 2; ++q) {
                         uint32_t r[32];
                         tmem_ld32(o_addr + 32u * q, r);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        for (int i = 0; i < 32; i += 2) {
+                            const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2);
+                            r[i] = __float_as_uint(o2.x);
+                            r[i + 1] = __float_as_uint(o2.y);
+                        }
                         tmem_st32(o_addr + 32u * q, r);
                     }
                     tmem_wait_st();
@@ -386,33 +436,41 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             tc_fence_before();
             mbar_arrive(smem_u32(&sm.bar_p_ready));
         }
-        if (ok && T > 0 &&
-            warp_wait(smem_u32(&sm.bar_o_done), (T - 1) & 1, abort_flag, p.status, limit)) {
-            tc_fence_after();
-            const float inv_l = 1.0f / l;
-            const uint32_t o_addr = tmem + lane_base + TM_O;
-            const int n = q0 + row;
-            const size_t orow = (size_t)bh * N + n;
+        if (ok && T > 0) {
+            // total row sum from both halves (the pair barrier's next phase)
+            const float l_half = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) + (lacc[2].x + lacc[2].y) +
+                                 (lacc[3].x + lacc[3].y);
+            sm.red_sum[half][row] = l_half;
+            mbar_arrive(smem_u32(&sm.bar_pair[quad][T & 1]));
+            ok = warp_wait(smem_u32(&sm.bar_pair[quad][T & 1]), (T >> 1) & 1, abort_flag, p.status, limit);
+            const float l = l_half + sm.red_sum[half ^ 1][row];
+            if (ok && warp_wait(smem_u32(&sm.bar_o_done), (T - 1) & 1, abort_flag, p.status, limit)) {
+                tc_fence_after();
+                const float inv_l = 1.0f / l;
+                const uint32_t o_addr = tmem + lane_base + TM_O + 64u * half;
+                const int n = q0 + row;
+                const size_t orow = (size_t)bh * N + n;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t r[32];
-                tmem_ld32(o_addr + 32u * q, r);
-                tmem_wait_ld();
-                if (n < N) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + 32 * q);
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t r[32];
+                    tmem_ld32(o_addr + 32u * q, r);
+                    tmem_wait_ld();
+                    if (n < N) {
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + 64 * half + 32 * q);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint32_t w[4];
+                        for (int v = 0; v < 4; ++v) {
+                            uint32_t w[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 8 * v + 2 * e;
-                            w[e] = pack_bf16x2(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l);
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 8 * v + 2 * e;
+                                w[e] = pack_bf16x2(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l);
+                            }
+                            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
+                if (p.lse && n < N && half == 0) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
             }
-            if (p.lse && n < N) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
         }
     }
 
@@ -430,8 +488,6 @@ struct ProbeSmem {
     uint8_t v[V_TILE_BYTES];
     uint8_t kc[CODE_TILE_BYTES];
     uint8_t qc[CODE_TILE_BYTES];
-    uint64_t ks_raw[128];
-    uint64_t qs_raw[128];
     uint8_t ks_atom[2][512];
     uint8_t qs_atom[2][512];
     uint64_t bar_full;
@@ -442,10 +498,9 @@ struct ProbeSmem {
 
 // mode 0: S = Qc Kc^T into out; mode 1: O = P V into out (P given in pbf).
 __global__ void __launch_bounds__(160, 1)
-    probe_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_qs,
-                 const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_ks,
-                 const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* pbf, float* out, int mode,
-                 int* status) {
+    probe_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_kc,
+                 const __grid_constant__ CUtensorMap tm_v, const uint64_t* q_scales, const uint64_t* k_scales,
+                 const __nv_bfloat16* pbf, float* out, int mode, int* status) {
     extern __shared__ uint8_t smem_raw[];
     ProbeSmem& sm = *align1024<ProbeSmem>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -465,13 +520,18 @@ __global__ void __launch_bounds__(160, 1)
     const uint32_t tmem = sm.tmem_base;
     volatile int* abort_flag = &sm.abort_flag;
     const uint32_t full = smem_u32(&sm.bar_full);
-    if (threadIdx.x == 0) {
+    if (mode == 0 && warp == 4) {
+        // the same scale staging as the attention kernel's producer warp
+        load_scale_atoms(q_scales, 128, sm.qs_atom[0], sm.qs_atom[1], lane);
+        load_scale_atoms(k_scales, 128, sm.ks_atom[0], sm.ks_atom[1], lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+    }
+    if (threadIdx.x == 128) {
         if (mode == 0) {
-            mbar_arrive_expect_tx(full, 2 * (CODE_TILE_BYTES + SCALE_TILE_BYTES));
+            mbar_arrive_expect_tx(full, 2 * CODE_TILE_BYTES);
             tma_load_3d(smem_u32(sm.qc), &tm_qc, 0, 0, 0, full);
-            tma_load_1d(smem_u32(sm.qs_raw), &tm_qs, 0, full);
             tma_load_3d(smem_u32(sm.kc), &tm_kc, 0, 0, 0, full);
-            tma_load_1d(smem_u32(sm.ks_raw), &tm_ks, 0, full);
         } else {
             mbar_arrive_expect_tx(full, V_TILE_BYTES);
             tma_load_3d(smem_u32(sm.v), &tm_v, 0, 0, 0, full);
@@ -499,12 +559,6 @@ __global__ void __launch_bounds__(160, 1)
     if (warp == 4) {
         ok = warp_wait(full, 0, abort_flag, status, kWaitLimitNs);
         if (ok) {
-            if (mode == 0) {
-                stage_scale_atoms(sm.qs_raw, sm.qs_atom[0], sm.qs_atom[1], lane);
-                stage_scale_atoms(sm.ks_raw, sm.ks_atom[0], sm.ks_atom[1], lane);
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
             if (lane == 0) {
                 tc_fence_after();
                 if (mode == 0) {
@@ -562,9 +616,10 @@ __global__ void wait_timeout_kernel(int* status, uint64_t limit_ns) {
 // ---------------------------------------------------------- host side ----
 
 struct Maps {
-    CUtensorMap qc, qs, kc, ks, v;
+    CUtensorMap qc, kc, v;
 };
 
+// Codes [BH][N][64 bytes]: 64B-swizzled boxes of 128 rows; x is always 0.
 bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N) {
     const uint64_t dims[3] = {64, (uint64_t)N, (uint64_t)BH};
     const uint64_t strides[2] = {64, (uint64_t)N * 64};
@@ -573,13 +628,8 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N) {
                              strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-bool make_scale_map(CUtensorMap* m, const uint8_t* base, int64_t rows) {
-    const uint64_t dims[1] = {(uint64_t)rows};
-    const uint32_t box[1] = {128};
-    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 1, const_cast<uint8_t*>(base), dims,
-                             nullptr, box, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
+// V [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x 128 keys; x is 0 or 64
+// (0 or 128 bytes), so every box starts on a 16-byte boundary.
 bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N) {
     const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH};
     const uint64_t strides[2] = {256, (uint64_t)N * 256};
@@ -597,8 +647,7 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     Maps m;
     if (!make_code_map(&m.qc, a.q_codes, a.BH, a.N) || !make_code_map(&m.kc, a.k_codes, a.BH, a.N) ||
-        !make_scale_map(&m.qs, a.q_scales, (int64_t)a.BH * a.N) ||
-        !make_scale_map(&m.ks, a.k_scales, (int64_t)a.BH * a.N) || !make_v_map(&m.v, a.v, a.BH, a.N))
+        !make_v_map(&m.v, a.v, a.BH, a.N))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(FwdSmem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = fwd_smem_bytes();
@@ -606,6 +655,8 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
         cudaSuccess)
         return FP4ATTN_ERR_CUDA;
     FwdParams p;
+    p.q_scales = reinterpret_cast<const uint64_t*>(a.q_scales);
+    p.k_scales = reinterpret_cast<const uint64_t*>(a.k_scales);
     p.N = a.N;
     p.n_kt = (a.N + BN - 1) / BN;
     const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 0.08838834764831845f;
@@ -617,7 +668,7 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;
     dim3 grid((a.N + BM - 1) / BM, a.BH);
-    fwd_kernel<<<grid, FWD_THREADS, smem, stream>>>(m.qc, m.qs, m.kc, m.ks, m.v, p);
+    fwd_kernel<<<grid, FWD_THREADS, smem, stream>>>(m.qc, m.kc, m.v, p);
     return cudaGetLastError() == cudaSuccess ? FP4ATTN_OK : FP4ATTN_ERR_CUDA;
 }
 
@@ -625,23 +676,19 @@ static int launch_probe(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc,
                         const __nv_bfloat16* p, const __nv_bfloat16* v, float* out, int mode,
                         cudaStream_t stream) {
     Maps m;
-    // Unused maps point at a valid operand of the same kind.
-    const uint8_t* qcb = qc ? qc : kc;
-    const uint8_t* qsb = qs ? qs : ks;
     if (mode == 0) {
-        if (!make_code_map(&m.qc, qcb, 1, 128) || !make_code_map(&m.kc, kc, 1, 128) ||
-            !make_scale_map(&m.qs, qsb, 128) || !make_scale_map(&m.ks, ks, 128))
-            return FP4ATTN_ERR_CUDA;
-        m.v = m.qc;
+        if (!make_code_map(&m.qc, qc, 1, 128) || !make_code_map(&m.kc, kc, 1, 128)) return FP4ATTN_ERR_CUDA;
+        m.v = m.qc;  // unused in this mode
     } else {
         if (!make_v_map(&m.v, v, 1, 128)) return FP4ATTN_ERR_CUDA;
-        m.qc = m.kc = m.qs = m.ks = m.v;
+        m.qc = m.kc = m.v;  // unused in this mode
     }
     const size_t smem = probe_smem_bytes();
     if (cudaFuncSetAttribute(probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return FP4ATTN_ERR_CUDA;
-    probe_kernel<<<1, 160, smem, stream>>>(m.qc, m.qs, m.kc, m.ks, m.v, p, out, mode, nullptr);
+    probe_kernel<<<1, 160, smem, stream>>>(m.qc, m.kc, m.v, reinterpret_cast<const uint64_t*>(qs),
+                                           reinterpret_cast<const uint64_t*>(ks), p, out, mode, nullptr);
     return cudaGetLastError() == cudaSuccess ? FP4ATTN_OK : FP4ATTN_ERR_CUDA;
 }
 

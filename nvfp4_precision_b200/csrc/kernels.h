@@ -9,9 +9,11 @@ namespace fp4attn {
 
 constexpr int D = 128;
 
-// Workspace layout: [0,256) status word and spare; [256, 256 + 8*BH*128)
-// int64 key column sums; then one uint32 per head (ready counters).
+// Workspace layout: [0,4) status word, [64,68) prologue tile ticket counter,
+// rest of [0,256) spare; [256, 256 + 8*BH*128) int64 key column sums; then
+// one uint32 per head (key-sum tiles completed).
 constexpr size_t WS_STATUS_BYTES = 256;
+constexpr size_t WS_TICKET_OFFSET = 64;
 inline size_t ws_ksum_offset() { return WS_STATUS_BYTES; }
 inline size_t ws_counter_offset(int64_t BH) { return WS_STATUS_BYTES + (size_t)BH * D * 8; }
 inline size_t ws_bytes(int64_t BH) {
@@ -33,6 +35,7 @@ struct QuantArgs {
     float* k_mean;  // may be nullptr
     long long* ksum;
     unsigned* counters;
+    unsigned* ticket;
     int* status;
 };
 

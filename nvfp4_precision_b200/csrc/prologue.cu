@@ -6,17 +6,25 @@
 // channels, fp32 per-tensor scale).  The fused transform there costs under
 // 1 ms per attention call on GB200.
 //
-// Two kernels, stream-ordered:
-//   ksum_kernel      exact int64 fixed-point column sums of K per head
-//                    (sum of round_half_even(k * 2^24)); order-independent,
-//                    so the atomics give the same bits as any serial order.
-//   quantize_kernel  one thread per 128-channel row: bf16 -> fp32, K minus the
-//                    head mean, 7 butterfly stages of ascending stride in
-//                    registers (no shuffles), x fp32(1/sqrt(128)), per-16 amax,
-//                    UE4M3 scale amax/6/g, E2M1 codes of y * (1/(g*scale)).
-// Every fp32 step is an explicit round-to-nearest intrinsic so nothing is
-// contracted into an FMA; the results are bit-identical to the plain CPU
-// definition of the same steps.
+// One persistent kernel.  CTAs take 128-row tiles from an atomic ticket queue
+// ordered per head as [key-sum tiles][Q tiles][K tiles]:
+//   key-sum tile   exact int64 fixed-point column sums of K (sum of
+//                  round_half_even(k * 2^24)); order-independent, so atomics
+//                  give the same bits as any serial order; then the head's
+//                  ready counter is bumped;
+//   Q / K tile     one thread per 128-channel row: bf16 -> fp32, (K) minus the
+//                  head mean once the head's counter is complete, the 7
+//                  butterfly stages of the Walsh-Hadamard transform in
+//                  registers, x fp32(1/sqrt(128)), per-16 amax, UE4M3 scale
+//                  amax/6/g, E2M1 codes of y * (1/(g*scale)).
+// The Q tiles of a head sit between its key-sum and K tiles, so the second
+// read of K mostly hits L2 (key-sum loads are marked evict-last, the others
+// evict-first).  Tiles arrive by TMA (128B swizzle) into a double buffer while
+// the previous tile is computed.  A row's 128 values live in registers as 64
+// pairs (x_i, x_{i+64}): the butterfly stages of stride 1..32 run on packed
+// fp32x2 instructions, the stride-64 stage inside each pair.  Every fp32 step
+// is an explicit round-to-nearest operation, so the codes are bit-identical to
+// the plain CPU definition of the same steps.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -28,207 +36,400 @@ namespace {
 
 constexpr float kTwo24 = 16777216.0f;
 constexpr float kKeyLimit = 1048576.0f;  // |k| < 2^20 keeps the int64 sum exact for N <= 2^18
-constexpr int KSUM_THREADS = 256;
-constexpr int KSUM_ROWS_PER_BLOCK = 2048;
+constexpr int PRO_THREADS = 128;         // one thread per row of a tile
+constexpr uint32_t HALF_BYTES = 128 * 128;        // 128 rows x 64 channels bf16
+constexpr uint32_t TILE_BYTES = 2 * HALF_BYTES;   // 32 KB
+constexpr uint64_t kSpinLimitNs = 2000000000ull;
+
+enum TileKind { KIND_KSUM = 0, KIND_Q = 1, KIND_K = 2 };
+
+struct __align__(1024) ProSmem {
+    uint8_t tile[2][TILE_BYTES];   // double buffer; channels 0-63 then 64-127, 128B swizzle
+    long long part[2][128];        // key-sum partials of even / odd rows
+    float2 neg_mean2[64];          // (-m_i, -m_{i+64})
+    float inv_scale[128];          // fp32 1 / value of each UE4M3 code (0 for code 0)
+    uint64_t bar[2];
+    int next_ticket[2];
+    int mean_head;
+    int abort_flag;
+};
+
+struct ProArgs {
+    uint8_t* codes[2];
+    uint8_t* scales[2];
+    const float* g[2];
+    long long* ksum;
+    unsigned* head_ready;
+    unsigned* ticket;
+    float* k_mean;
+    int BH, N, n_tiles;
+    uint32_t flags;
+    int* status;
+};
 
 __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
-// ----------------------------------------------------------- key sums -----
-
-// grid (ceil(N / KSUM_ROWS_PER_BLOCK), BH); 16 threads per row (8 channels
-// each, one 16-byte load), 16 rows in flight per block iteration.
-__global__ void __launch_bounds__(KSUM_THREADS) ksum_kernel(const __nv_bfloat16* __restrict__ k,
-                                                            int N, long long* __restrict__ ksum,
-                                                            int* status) {
-    const int bh = blockIdx.y;
-    const int n0 = blockIdx.x * KSUM_ROWS_PER_BLOCK;
-    const int n1 = min(N, n0 + KSUM_ROWS_PER_BLOCK);
-    const int cg = threadIdx.x & 15;   // channel group: channels 8cg .. 8cg+7
-    const int rg = threadIdx.x >> 4;   // row group 0..15
-    long long acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0;
-    bool bad = false;
-    const uint4* base = reinterpret_cast<const uint4*>(k + ((size_t)bh * N) * D) + cg;
-    for (int n = n0 + rg; n < n1; n += 16) {
-        const uint4 raw = __ldg(base + (size_t)n * (D / 8));
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float v = (e & 1) ? bf16hi(w[e >> 1]) : bf16lo(w[e >> 1]);
-            if (fabsf(v) < kKeyLimit) {
-                acc[e] += __float2ll_rn(__fmul_rn(v, kTwo24));  // exact product, ties-to-even
-            } else {
-                bad = true;  // also catches NaN
-            }
-        }
-    }
-    __shared__ long long part[16][D];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) part[rg][cg * 8 + e] = acc[e];
-    __syncthreads();
-    if (threadIdx.x < D) {
-        long long t = 0;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) t += part[r][threadIdx.x];
-        atomicAdd(reinterpret_cast<unsigned long long*>(ksum + (size_t)bh * D + threadIdx.x),
-                  static_cast<unsigned long long>(t));
-    }
-    if (bad) set_status(status, FP4ATTN_ERR_RANGE);
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
-// ----------------------------------------------------------- transform -----
-
-// Unnormalised Sylvester Walsh-Hadamard transform, butterflies of stride
-// 1, 2, ..., 64 in that order.
-__device__ __forceinline__ void fwht128(float (&x)[D]) {
-#pragma unroll
-    for (int h = 1; h < D; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < D; ++i) {
-            if ((i & h) == 0) {
-                const float a = x[i], b = x[i + h];
-                x[i] = __fadd_rn(a, b);
-                x[i + h] = __fsub_rn(a, b);
-            }
-        }
-    }
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                 int32_t c2, uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
+        : "memory");
 }
 
-// NVFP4 pack of one 16-value block: two code words (element 0 in the low
-// nibble of word0) and the UE4M3 scale byte.
-__device__ __forceinline__ void pack_block(const float* y, float g, bool g_is_one, uint32_t& w0,
-                                           uint32_t& w1, uint32_t& scale) {
-    float a = 0.0f;
+// Byte offset of 16-byte chunk j (0..7) of row r inside one 128B-swizzled
+// half tile: the chunk index is XORed with the row index mod 8, which also
+// makes eight consecutive rows reading the same chunk hit distinct banks.
+__device__ __forceinline__ uint32_t swz(int r, int j) { return (uint32_t)r * 128u + ((uint32_t)(j ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, f2(-1.0f, -1.0f), a); }
+
+__device__ __forceinline__ float amax16(const float2* p, bool hi) {
+    float a[6];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(y[i]));
+    for (int k = 0; k < 5; ++k) {
+        const float x0 = hi ? p[3 * k].y : p[3 * k].x;
+        const float x1 = hi ? p[3 * k + 1].y : p[3 * k + 1].x;
+        const float x2 = hi ? p[3 * k + 2].y : p[3 * k + 2].x;
+        a[k] = fmax3(fabsf(x0), fabsf(x1), fabsf(x2));
+    }
+    a[5] = fabsf(hi ? p[15].y : p[15].x);
+    return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), 0.0f);
+}
+
+// Scale byte and 1/(g*scale) of one block with amax a.
+__device__ __forceinline__ void block_scale(float a, float g, bool g_is_one, const float* inv_tab, uint32_t& s,
+                                            float& inv) {
     float t = __fdiv_rn(a, 6.0f);
     if (!g_is_one) t = __fdiv_rn(t, g);
-    const uint32_t s = cvt_e4m3(t);  // t >= 0: the E4M3 byte is the UE4M3 byte
-    const float sd = ue4m3_value(s);
-    float inv = 0.0f;
-    if (sd != 0.0f) inv = __frcp_rn(g_is_one ? sd : __fmul_rn(g, sd));
-    float r[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) r[i] = __fmul_rn(y[i], inv);
-    w0 = cvt_e2m1x8(r[0], r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
-    w1 = cvt_e2m1x8(r[8], r[9], r[10], r[11], r[12], r[13], r[14], r[15]);
-    scale = s;
+    s = cvt_e4m3(t);  // t >= +0: the E4M3 byte is the UE4M3 byte
+    if (g_is_one) {
+        inv = inv_tab[s];
+    } else {
+        const float sd = ue4m3_value(s);
+        inv = (sd != 0.0f) ? __frcp_rn(__fmul_rn(g, sd)) : 0.0f;
+    }
 }
 
-struct QuantKernelArgs {
-    const __nv_bfloat16* src[2];  // Q, K
-    uint8_t* codes[2];
-    uint8_t* scales[2];
-    const float* g[2];
-    const long long* ksum;
-    float* k_mean;
-    int N;
-    uint32_t flags;
-    int* status;
-};
-
-constexpr int QUANT_ROWS = 128;
-
-// grid (ceil(N / 128), BH, 2): z = 0 quantises Q rows, z = 1 K rows.  One
-// thread per row.
-__global__ void __launch_bounds__(QUANT_ROWS) quantize_kernel(const QuantKernelArgs a) {
-    const int which = blockIdx.z;
-    const int bh = blockIdx.y;
+__global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                               const __grid_constant__ CUtensorMap tm_k,
+                                                               const ProArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    ProSmem& sm = *reinterpret_cast<ProSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
     const int N = a.N;
-    const int n = blockIdx.x * QUANT_ROWS + threadIdx.x;
-    const bool smooth = (which == 1) && !(a.flags & FP4ATTN_NO_SMOOTH_K);
+    const int Th = a.n_tiles;
+    const bool smooth = !(a.flags & FP4ATTN_NO_SMOOTH_K);
     const bool hadamard = !(a.flags & FP4ATTN_NO_HADAMARD);
+    const int per_head = (smooth ? 3 : 2) * Th;
+    const int total = a.BH * per_head;
 
-    __shared__ float mean_s[D];
-    if (smooth) {
-        const int c = threadIdx.x;  // blockDim.x == D
-        const double num = __ll2double_rn(a.ksum[(size_t)bh * D + c]);
-        const double den = (double)N * 16777216.0;
-        const float m = __double2float_rn(__ddiv_rn(num, den));
-        mean_s[c] = m;
-        if (a.k_mean && blockIdx.x == 0) a.k_mean[(size_t)bh * D + c] = m;
-    } else if (which == 1 && a.k_mean && blockIdx.x == 0) {
-        a.k_mean[(size_t)bh * D + threadIdx.x] = 0.0f;
+    if (tid == 0) {
+        mbar_init(smem_u32(&sm.bar[0]), 1);
+        mbar_init(smem_u32(&sm.bar[1]), 1);
+        sm.mean_head = -1;
+        sm.abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+    }
+    {
+        const float sd = ue4m3_value(tid);  // tid < 128 covers every code; 127 (NaN) is never produced
+        sm.inv_scale[tid] = (sd != 0.0f) ? __frcp_rn(sd) : 0.0f;
+    }
+    float g[2] = {1.0f, 1.0f};
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        if (a.g[w]) {
+            g[w] = *a.g[w];
+            if (!(g[w] > 0.0f && g[w] < INFINITY) && tid == 0) set_status(a.status, FP4ATTN_ERR_RANGE);
+        }
     }
     __syncthreads();
 
-    float g = 1.0f;
-    if (a.g[which]) {
-        g = *a.g[which];
-        if (!(g > 0.0f && g < INFINITY)) set_status(a.status, FP4ATTN_ERR_RANGE);
-    }
-    const bool g_is_one = (g == 1.0f);
-    if (n >= N) return;
+    const uint64_t pol_keep = l2_policy_evict_last();
+    const uint64_t pol_stream = l2_policy_evict_first();
+    auto decode = [&](int t, int& kind, int& bh, int& tile) {
+        bh = t / per_head;
+        const int l = t - bh * per_head;
+        kind = (smooth ? 0 : 1) + l / Th;
+        tile = l % Th;
+    };
+    auto issue = [&](int t, int buf) {  // thread 0 only
+        int kind, bh, tile;
+        decode(t, kind, bh, tile);
+        const CUtensorMap* map = (kind == KIND_Q) ? &tm_q : &tm_k;
+        const uint64_t pol = (kind == KIND_KSUM) ? pol_keep : pol_stream;
+        const uint32_t bar = smem_u32(&sm.bar[buf]);
+        mbar_arrive_expect_tx(bar, TILE_BYTES);
+        tma_load_3d_hint(smem_u32(sm.tile[buf]), map, 0, tile * 128, bh, bar, pol);
+        tma_load_3d_hint(smem_u32(sm.tile[buf]) + HALF_BYTES, map, 64, tile * 128, bh, bar, pol);
+    };
 
-    const size_t row = (size_t)bh * N + n;
-    const uint4* src = reinterpret_cast<const uint4*>(a.src[which] + row * D);
-    float x[D];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-        const uint4 raw = __ldg(src + i);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[8 * i + e] = (e & 1) ? bf16hi(w[e >> 1]) : bf16lo(w[e >> 1]);
+    bool in_flight[2] = {false, false};  // tracked by thread 0, which issues the copies
+    if (tid == 0) {
+        const int t0 = (int)atomicAdd(a.ticket, 1u);
+        sm.next_ticket[0] = t0;
+        if (t0 < total) {
+            issue(t0, 0);
+            in_flight[0] = true;
+        }
     }
-    bool finite = true;
-#pragma unroll
-    for (int i = 0; i < D; ++i) finite &= (fabsf(x[i]) < INFINITY);
-    if (!finite) set_status(a.status, FP4ATTN_ERR_RANGE);
+    __syncthreads();
+    int t = sm.next_ticket[0];
+    int buf = 0;
+    uint32_t phase[2] = {0u, 0u};
 
-    if (smooth) {
+    while (t < total) {
+        // prefetch the next tile into the other buffer
+        if (tid == 0) {
+            const int tn = (int)atomicAdd(a.ticket, 1u);
+            sm.next_ticket[buf ^ 1] = tn;
+            if (tn < total) {
+                issue(tn, buf ^ 1);
+                in_flight[buf ^ 1] = true;
+            }
+        }
+        int kind, bh, tile;
+        decode(t, kind, bh, tile);
+        const bool landed = mbar_wait(smem_u32(&sm.bar[buf]), phase[buf], &sm.abort_flag, a.status, kSpinLimitNs);
+        if (__syncthreads_or(!landed)) break;
+        phase[buf] ^= 1u;
+        in_flight[buf] = false;
+        const uint8_t* tb = sm.tile[buf];
+
+        if (kind == KIND_KSUM) {
+            // ------------------------------------------------ key sums ----
+            const int cp = tid & 63;       // channel pair (2cp, 2cp+1)
+            const int rpar = tid >> 6;     // rows of this parity
+            const uint8_t* hb = tb + (cp >> 5) * HALF_BYTES;
+            const int j = (cp & 31) >> 2;
+            const uint32_t in_chunk = (uint32_t)(cp & 3) * 4u;
+            long long acc0 = 0, acc1 = 0;
+            bool bad = false;
+#pragma unroll 8
+            for (int r = rpar; r < 128; r += 2) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(hb + swz(r, j) + in_chunk);
+                const float v0 = bf16lo(w), v1 = bf16hi(w);
+                if (fabsf(v0) < kKeyLimit) acc0 += __float2ll_rn(__fmul_rn(v0, kTwo24)); else bad = true;
+                if (fabsf(v1) < kKeyLimit) acc1 += __float2ll_rn(__fmul_rn(v1, kTwo24)); else bad = true;
+            }
+            if (bad) set_status(a.status, FP4ATTN_ERR_RANGE);
+            sm.part[rpar][2 * cp] = acc0;
+            sm.part[rpar][2 * cp + 1] = acc1;
+            __syncthreads();
+            const long long tot = sm.part[0][tid] + sm.part[1][tid];
+            atomicAdd(reinterpret_cast<unsigned long long*>(a.ksum + (size_t)bh * D + tid),
+                      static_cast<unsigned long long>(tot));
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicAdd(a.head_ready + bh, 1u);
+        } else {
+            const int which = kind - 1;  // 0 = Q, 1 = K
+            if (which == 1 && sm.mean_head != bh) {
+                // ------------------------------------------ head means ----
+                bool ready = true;
+                if (smooth && tid == 0) {
+                    volatile unsigned* cnt = a.head_ready + bh;
+                    const uint64_t t0 = globaltimer_ns();
+                    while (*cnt < (unsigned)Th) {
+                        if (globaltimer_ns() - t0 > kSpinLimitNs) {
+                            set_status(a.status, FP4ATTN_ERR_TIMEOUT);
+                            ready = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    __threadfence();
+                }
+                if (__syncthreads_or(!ready)) break;
+                float m = 0.0f;
+                if (smooth) {
+                    const long long S = __ldcg(a.ksum + (size_t)bh * D + tid);
+                    m = __double2float_rn(__ddiv_rn(__ll2double_rn(S), (double)N * 16777216.0));
+                }
+                if (tid < 64) sm.neg_mean2[tid].x = -m; else sm.neg_mean2[tid - 64].y = -m;
+                if (a.k_mean && tile == 0) a.k_mean[(size_t)bh * D + tid] = m;
+                __syncthreads();
+                if (tid == 0) sm.mean_head = bh;
+            }
+            // ---------------------------------------------- one row ----
+            const int r = tid;
+            float2 P[64];  // P[i] = (x_i, x_{i+64})
+            const bool sub_mean = (which == 1) && smooth;
+            bool finite = true;
+            // chunk j holds pairs 8j..8j+7: load, unpack, smooth, and apply the
+            // butterfly stages of stride 1, 2, 4, which stay inside the chunk
 #pragma unroll
-        for (int i = 0; i < D; ++i) x[i] = __fsub_rn(x[i], mean_s[i]);
+            for (int j = 0; j < 8; ++j) {
+                const uint4 lo = *reinterpret_cast<const uint4*>(tb + swz(r, j));
+                const uint4 hi = *reinterpret_cast<const uint4*>(tb + HALF_BYTES + swz(r, j));
+                const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
+                const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
+                float2* C = P + 8 * j;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    C[2 * e] = f2(bf16lo(wl[e]), bf16lo(wh[e]));
+                    C[2 * e + 1] = f2(bf16hi(wl[e]), bf16hi(wh[e]));
+                }
+                if (sub_mean) {
+                    const float4* nm = reinterpret_cast<const float4*>(sm.neg_mean2 + 8 * j);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 m4 = nm[e];
+                        C[2 * e] = __fadd2_rn(C[2 * e], f2(m4.x, m4.y));
+                        C[2 * e + 1] = __fadd2_rn(C[2 * e + 1], f2(m4.z, m4.w));
+                    }
+                }
+                if (!hadamard) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) finite &= (fabsf(C[i].x) < INFINITY) && (fabsf(C[i].y) < INFINITY);
+                } else {
+#pragma unroll
+                    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            if ((i & h) == 0) {
+                                const float2 x = C[i], y = C[i + h];
+                                C[i] = __fadd2_rn(x, y);
+                                C[i + h] = sub2(x, y);
+                            }
+                        }
+                    }
+                }
+            }
+            if (hadamard) {
+                // strides 8, 16, 32 across chunks, then 64 inside each pair
+#pragma unroll
+                for (int h = 8; h < 64; h <<= 1) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        if ((i & h) == 0) {
+                            const float2 x = P[i], y = P[i + h];
+                            P[i] = __fadd2_rn(x, y);
+                            P[i + h] = sub2(x, y);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 64; ++i) P[i] = f2(__fadd_rn(P[i].x, P[i].y), __fsub_rn(P[i].x, P[i].y));
+                // y_0 is the sum of all 128 inputs: it is finite iff they all are
+                // (barring overflow of the sum itself)
+                finite = fabsf(P[0].x) < INFINITY;
+                const float c = __uint_as_float(0x3DB504F3u);  // fp32(1/sqrt(128))
+#pragma unroll
+                for (int i = 0; i < 64; ++i) P[i] = __fmul2_rn(P[i], f2(c, c));
+            }
+
+            // NVFP4 pack.  Blocks 0-3 are the .x lanes of P[0..63], blocks 4-7
+            // the .y lanes; block b's codes are words 2b, 2b+1 of the row.
+            const float gw = g[which];
+            const bool g_is_one = (gw == 1.0f);
+            const bool valid = (tile * 128 + r) < N;
+            if (!finite && valid) set_status(a.status, FP4ATTN_ERR_RANGE);
+            const size_t row = (size_t)bh * N + (size_t)tile * 128 + r;
+            uint4* dst = reinterpret_cast<uint4*>(a.codes[which] + row * 64);
+            uint32_t lo[4], hi[4];  // code words of blocks (bb-1, bb) and (bb+3, bb+4)
+            uint32_t sw_lo = 0, sw_hi = 0;
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                uint32_t s_lo, s_hi;
+                float inv_lo, inv_hi;
+                block_scale(amax16(P + 16 * bb, false), gw, g_is_one, sm.inv_scale, s_lo, inv_lo);
+                block_scale(amax16(P + 16 * bb, true), gw, g_is_one, sm.inv_scale, s_hi, inv_hi);
+                sw_lo |= s_lo << (8 * bb);
+                sw_hi |= s_hi << (8 * bb);
+                const float2 inv2 = f2(inv_lo, inv_hi);
+#pragma unroll
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    float2 R[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) R[k] = __fmul2_rn(P[16 * bb + 8 * h8 + k], inv2);
+                    lo[2 * (bb & 1) + h8] = cvt_e2m1x8(R[0].x, R[1].x, R[2].x, R[3].x, R[4].x, R[5].x, R[6].x, R[7].x);
+                    hi[2 * (bb & 1) + h8] = cvt_e2m1x8(R[0].y, R[1].y, R[2].y, R[3].y, R[4].y, R[5].y, R[6].y, R[7].y);
+                }
+                if ((bb & 1) && valid) {
+                    dst[bb >> 1] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    dst[2 + (bb >> 1)] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                }
+            }
+            if (valid) *reinterpret_cast<uint2*>(a.scales[which] + row * 8) = make_uint2(sw_lo, sw_hi);
+        }
+        __syncthreads();  // tile[buf] is free; next_ticket[buf ^ 1] is visible
+        t = sm.next_ticket[buf ^ 1];
+        buf ^= 1;
     }
-    if (hadamard) {
-        fwht128(x);
-        const float c = __uint_as_float(0x3DB504F3u);  // fp32(1/sqrt(128))
-#pragma unroll
-        for (int i = 0; i < D; ++i) x[i] = __fmul_rn(x[i], c);
+    // wind down after an abort: let this CTA's own copies land before exiting
+    if (tid == 0) {
+        int dummy = 0;
+        for (int b = 0; b < 2; ++b)
+            if (in_flight[b]) mbar_wait(smem_u32(&sm.bar[b]), phase[b], &dummy, nullptr, 200000000ull);
     }
+}
 
-    uint32_t cw[16];
-    uint32_t sb[8];
-#pragma unroll
-    for (int b = 0; b < 8; ++b) pack_block(x + 16 * b, g, g_is_one, cw[2 * b], cw[2 * b + 1], sb[b]);
+size_t pro_smem_bytes() { return sizeof(ProSmem) + 1024; }
 
-    uint4* dst = reinterpret_cast<uint4*>(a.codes[which] + row * 64);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
-    uint2 s2;
-    s2.x = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
-    s2.y = sb[4] | (sb[5] << 8) | (sb[6] << 16) | (sb[7] << 24);
-    *reinterpret_cast<uint2*>(a.scales[which] + row * 8) = s2;
+bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N) {
+    // [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x 128 rows; x is 0 or 64
+    // (0 or 128 bytes), so every box starts on a 16-byte boundary.
+    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH};
+    const uint64_t strides[2] = {256, (uint64_t)N * 256};
+    const uint32_t box[3] = {64, 128, 1};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(base), dims,
+                             strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
 
-cudaError_t launch_quantize_qk(const QuantArgs& a, cudaStream_t stream) {
-    if (a.BH == 0 || a.N == 0) return cudaSuccess;
-    if (!(a.flags & FP4ATTN_NO_SMOOTH_K)) {
-        dim3 grid((a.N + KSUM_ROWS_PER_BLOCK - 1) / KSUM_ROWS_PER_BLOCK, a.BH);
-        ksum_kernel<<<grid, KSUM_THREADS, 0, stream>>>(a.k, a.N, a.ksum, a.status);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    QuantKernelArgs k{};
-    k.src[0] = a.q;
-    k.src[1] = a.k;
-    k.codes[0] = a.q_codes;
-    k.codes[1] = a.k_codes;
-    k.scales[0] = a.q_scales;
-    k.scales[1] = a.k_scales;
-    k.g[0] = a.gq;
-    k.g[1] = a.gk;
-    k.ksum = a.ksum;
-    k.k_mean = a.k_mean;
-    k.N = a.N;
-    k.flags = a.flags;
-    k.status = a.status;
-    dim3 grid((a.N + QUANT_ROWS - 1) / QUANT_ROWS, a.BH, 2);
-    quantize_kernel<<<grid, QUANT_ROWS, 0, stream>>>(k);
+cudaError_t launch_quantize_qk(const QuantArgs& q, cudaStream_t stream) {
+    if (q.BH == 0 || q.N == 0) return cudaSuccess;
+    CUtensorMap tm_q, tm_k;
+    if (!make_rows_map(&tm_q, q.q, q.BH, q.N) || !make_rows_map(&tm_k, q.k, q.BH, q.N)) return cudaErrorInvalidValue;
+    static_assert(sizeof(ProSmem) + 1024 <= 227 * 1024, "shared memory budget");
+    const size_t smem = pro_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prologue_kernel, PRO_THREADS, smem)) !=
+        cudaSuccess)
+        return e;
+    ProArgs a{};
+    a.codes[0] = q.q_codes;
+    a.codes[1] = q.k_codes;
+    a.scales[0] = q.q_scales;
+    a.scales[1] = q.k_scales;
+    a.g[0] = q.gq;
+    a.g[1] = q.gk;
+    a.ksum = q.ksum;
+    a.head_ready = q.counters;
+    a.ticket = q.ticket;
+    a.k_mean = q.k_mean;
+    a.BH = q.BH;
+    a.N = q.N;
+    a.n_tiles = (q.N + 127) / 128;
+    a.flags = q.flags;
+    a.status = q.status;
+    const long long tiles = (long long)a.BH * a.n_tiles * ((q.flags & FP4ATTN_NO_SMOOTH_K) ? 2 : 3);
+    long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
+    if (grid > tiles) grid = tiles;
+    prologue_kernel<<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, a);
     return cudaGetLastError();
 }
 

@@ -71,15 +71,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // -------------------------------------------------------------------- TMA --
 
-__device__ __forceinline__ void tma_load_1d(uint32_t dst, const CUtensorMap* map, int32_t c0,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2}], [%3];" ::"r"(dst),
-        "l"(map), "r"(c0), "r"(bar)
-        : "memory");
-}
-
+// 3-D tiled bulk tensor copy global -> shared.  The innermost coordinate times
+// the element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t c0,
                                             int32_t c1, int32_t c2, uint32_t bar) {
     asm volatile(
@@ -278,6 +271,33 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of values on the FMA pipe (no MUFU).  Cody-Waite range
+// reduction x = n + f with n = rn(x), f in [-1/2, 1/2]: adding 1.5 * 2^23
+// rounds x to an integer held in the low mantissa bits of t (Schraudolph's
+// shifter), 2^f is a degree-3 minimax polynomial (relative error 1.0e-4,
+// fitted by gen_exp2_poly.py --half), and n is added to the exponent field
+// by shifting t's mantissa bits into place.  Inputs below -125 are clamped
+// there (the result is then below 2^-124).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+    float2 acc = __ffma2_rn(make_float2(0.055009543895721436f, 0.055009543895721436f), f,
+                            make_float2(0.24221102893352509f, 0.24221102893352509f));
+    acc = __ffma2_rn(acc, f, make_float2(0.6932827830314636f, 0.6932827830314636f));
+    acc = __ffma2_rn(acc, f, make_float2(1.0f, 1.0f));
+    return make_float2(__int_as_float(__float_as_int(acc.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(acc.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace fp4attn
