@@ -109,6 +109,33 @@ int fp4attn_forward(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
                     void* o_bf16_dev, float* lse_dev,
                     void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
 
+/* fp4attn_quantize_qk without a workspace argument.  The pages have no
+ * counterpart to this entry point: it exists for callers that cannot allocate
+ * device memory for the workspace -- cudaMalloc/cudaFree may synchronise the
+ * whole device, which a latency-bound caller sharing the GPU cannot afford,
+ * and some callers run where another allocator owns all device memory and
+ * raw allocations are not allowed.  It allocates nothing: its scratch (status
+ * word, ticket, key sums) is a fixed array of about 1 MB in the library's
+ * device memory, held by every GPU that loads the library until the process
+ * exits.  The caller still passes every input and output, as for
+ * fp4attn_quantize_qk, whose arguments and results this call shares.
+ *   status_dev : device int32 that receives the device status word of this
+ *     call (FP4ATTN_OK or the first device error), or NULL.
+ * Limits and behaviour:
+ *   - B*H at most 1024; larger shapes return FP4ATTN_ERR_UNSUPPORTED and
+ *     launch nothing;
+ *   - the first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture;
+ *   - every call shares the one array and clears what must start at zero on
+ *     its stream; calls that overlap on the GPU (other streams, other host
+ *     threads) race on it and must be serialised by the caller. */
+int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, fp4attn_shape s,
+                                const float* q_gscale_dev, const float* k_gscale_dev, uint32_t flags,
+                                uint8_t* q_codes_dev, uint8_t* q_scales_dev,
+                                uint8_t* k_codes_dev, uint8_t* k_scales_dev, float* k_mean_dev,
+                                int* status_dev, cudaStream_t stream);
+
 /* Testing: decode NVFP4 rows back to fp32, out = fl(fl(g * s) * e2m1).
  *   codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or NULL,
  *   out_dev fp32 [rows,128], rows = B*H*N of s. */

@@ -27,7 +27,8 @@ NO_SMOOTH_K = 1
 NO_HADAMARD = 2
 
 EXPORTS = (
-    "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_forward", "fp4attn_dequant",
+    "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_quantize_qk_noalloc", "fp4attn_forward",
+    "fp4attn_dequant",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
 )
@@ -53,6 +54,8 @@ def _load():
     L.fp4attn_workspace_bytes.argtypes = [Shape]
     L.fp4attn_quantize_qk.restype = ctypes.c_int
     L.fp4attn_quantize_qk.argtypes = [P, P, Shape, P, P, U32, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_quantize_qk_noalloc.restype = ctypes.c_int
+    L.fp4attn_quantize_qk_noalloc.argtypes = [P, P, Shape, P, P, U32, P, P, P, P, P, P, P]
     L.fp4attn_forward.restype = ctypes.c_int
     L.fp4attn_forward.argtypes = [P, P, P, P, P, P, P, Shape, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
     L.fp4attn_dequant.restype = ctypes.c_int
@@ -134,6 +137,33 @@ def fp4attn_quantize_qk(q: torch.Tensor, k: torch.Tensor, q_gscale: Optional[tor
                                  workspace.numel(), _stream(stream))
     _check(rc, "fp4attn_quantize_qk")
     out["workspace"] = workspace
+    return out
+
+
+def fp4attn_quantize_qk_noalloc(q: torch.Tensor, k: torch.Tensor, q_gscale: Optional[torch.Tensor] = None,
+                                k_gscale: Optional[torch.Tensor] = None, flags: int = 0, out: Optional[dict] = None,
+                                k_mean: bool = True, status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """fp4attn_quantize_qk for callers that cannot allocate a workspace: the
+    library's fixed scratch array is used instead (B*H <= 1024).  The outputs
+    (and the optional int32 ``status`` tensor receiving the device status)
+    are the caller's.  Returns dict(q_codes, q_scales, k_codes, k_scales,
+    k_mean, status)."""
+    assert q.dtype == torch.bfloat16 and k.dtype == torch.bfloat16 and q.shape == k.shape
+    assert q.is_contiguous() and k.is_contiguous()
+    B, H, N, D = q.shape
+    dev = q.device
+    if out is None:
+        out = dict(q_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
+                   q_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
+                   k_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
+                   k_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
+                   k_mean=torch.empty((B, H, 128), dtype=torch.float32, device=dev) if k_mean else None)
+    rc = lib.fp4attn_quantize_qk_noalloc(_ptr(q), _ptr(k), Shape(B, H, N, D), _ptr(q_gscale), _ptr(k_gscale),
+                                         int(flags), _ptr(out["q_codes"]), _ptr(out["q_scales"]),
+                                         _ptr(out["k_codes"]), _ptr(out["k_scales"]), _ptr(out.get("k_mean")),
+                                         _ptr(status), _stream(stream))
+    _check(rc, "fp4attn_quantize_qk_noalloc")
+    out["status"] = status
     return out
 
 
