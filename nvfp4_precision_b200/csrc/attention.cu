@@ -4,15 +4,17 @@
 // Method: FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention":
 // queries and keys are quantised for an NVFP4 attention kernel; P and V stay
 // in BF16.  This kernel is written for sm_100a:
-//   * one CTA per (head, 128-query tile); 320 threads in three roles
-//       warps 0-7  softmax, O correction and epilogue; query row r is TMEM
-//                  lane r and is shared by warps r/32 (keys 0-63 of each
-//                  tile) and r/32 + 4 (keys 64-127), which exchange their
-//                  partial row maxima through shared memory every tile;
-//       warp 8     producer: scale-factor atoms (plain loads) and TMA copies
-//                  of Q once, then K codes and V tiles of 128 keys into a
+//   * one CTA per (head, 128-query tile); 4 * COL_GROUPS softmax warps plus
+//     two more:
+//       softmax    softmax, O correction and epilogue; query row r is TMEM
+//                  lane r and is shared by the COL_GROUPS warps w with
+//                  w % 4 == r / 32, each owning 128 / COL_GROUPS key columns
+//                  of every tile; they exchange partial row maxima through
+//                  shared memory every tile;
+//       producer   scale-factor atoms (plain loads) and TMA copies of Q
+//                  once, then K codes and V tiles of 128 keys into a
 //                  STAGES-deep shared-memory ring;
-//       warp 9     TMEM owner and MMA issuer: stages the scale factors into
+//       MMA        TMEM owner and MMA issuer: stages the scale factors into
 //                  TMEM (tcgen05.cp) and issues S = Q K^T with
 //                  tcgen05.mma kind::mxf4nvf4 (block16 scales) and
 //                  O += P V with tcgen05.mma kind::f16 (P read from TMEM);
@@ -38,14 +40,26 @@ namespace {
 
 constexpr int BM = 128;  // query rows per CTA
 constexpr int BN = 128;  // keys per tile
-constexpr int STAGES = 3;
-constexpr int SOFTMAX_WARPS = 8;
+constexpr int STAGES = 4;
+// Softmax warps come in COL_GROUPS groups of four (one warp per TMEM
+// sub-partition); each warp owns CW of the 128 score columns of its 32 rows.
+#ifndef FP4ATTN_COL_GROUPS
+#define FP4ATTN_COL_GROUPS 2
+#endif
+// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
+// and the rest to MUFU ex2 (MUFU issues 16 per clock per SM).
+#ifndef FP4ATTN_POLY_PAIRS
+#define FP4ATTN_POLY_PAIRS 3
+#endif
+constexpr int COL_GROUPS = FP4ATTN_COL_GROUPS;
+static_assert(COL_GROUPS == 2 || COL_GROUPS == 4, "2 or 4 column groups");
+constexpr int CW = 128 / COL_GROUPS;  // score columns per softmax warp
+constexpr int CW32 = CW / 32;         // 32-column TMEM loads per tile
+constexpr int SOFTMAX_WARPS = 4 * COL_GROUPS;
 constexpr int FWD_THREADS = 32 * (SOFTMAX_WARPS + 2);
 constexpr int WARP_PRODUCER = SOFTMAX_WARPS;
 constexpr int WARP_MMA = SOFTMAX_WARPS + 1;
-// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
-// and the rest to MUFU ex2 (MUFU issues 16 per clock per SM).
-constexpr int POLY_PAIRS_PER_8 = 3;
+constexpr int POLY_PAIRS_PER_8 = FP4ATTN_POLY_PAIRS;
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0;
@@ -76,12 +90,13 @@ struct __align__(1024) FwdSmem {
     uint64_t bar_kv_full[STAGES];
     uint64_t bar_kv_empty[STAGES];
     uint64_t bar_s_full[2];
-    uint64_t bar_p_ready;
-    uint64_t bar_o_done;
+    uint64_t bar_p_ready[2];      // P of tiles with this parity is in TMEM
+    uint64_t bar_o_done;          // O holds the P.V of every tile up to the last commit
+    uint64_t bar_o_final;         // the last tile's P.V is done
     uint64_t bar_final;
-    uint64_t bar_pair[4][2];      // per row quarter, per tile parity: both halves' maxima are in
-    float red_max[2][2][128];     // [tile parity][half][row] partial row maxima
-    float red_sum[2][128];        // [half][row] partial row sums, at the end
+    uint64_t bar_group[4][2];              // per sub-partition, per tile parity: all partial maxima are in
+    float red_max[2][COL_GROUPS][128];     // [tile parity][column group][row] partial row maxima
+    float red_sum[COL_GROUPS][128];        // [column group][row] partial row sums, at the end
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -128,18 +143,26 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
 // sub-partition.  One full warp, lane = line; rows at or beyond n_rows read
 // as zero.  Plain 8-byte loads: a row's scales start at any multiple of 8
 // bytes, which a bulk tensor copy could not address.
-__device__ __forceinline__ void load_scale_atoms(const uint64_t* rows, int n_rows, uint8_t* atom0,
-                                                 uint8_t* atom1, int lane) {
-    uint32_t lo[4], hi[4];
+__device__ __forceinline__ void fetch_scales(const uint64_t* rows, int n_rows, int lane, uint64_t (&w)[4]) {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const int r = lane + 32 * c;
-        const uint64_t w = (r < n_rows) ? __ldg(reinterpret_cast<const unsigned long long*>(rows) + r) : 0ull;
-        lo[c] = (uint32_t)w;
-        hi[c] = (uint32_t)(w >> 32);
+        w[c] = (r < n_rows) ? __ldg(reinterpret_cast<const unsigned long long*>(rows) + r) : 0ull;
     }
-    *reinterpret_cast<uint4*>(atom0 + 16 * lane) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    *reinterpret_cast<uint4*>(atom1 + 16 * lane) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+}
+
+__device__ __forceinline__ void store_scale_atoms(const uint64_t (&w)[4], uint8_t* atom0, uint8_t* atom1, int lane) {
+    *reinterpret_cast<uint4*>(atom0 + 16 * lane) =
+        make_uint4((uint32_t)w[0], (uint32_t)w[1], (uint32_t)w[2], (uint32_t)w[3]);
+    *reinterpret_cast<uint4*>(atom1 + 16 * lane) =
+        make_uint4((uint32_t)(w[0] >> 32), (uint32_t)(w[1] >> 32), (uint32_t)(w[2] >> 32), (uint32_t)(w[3] >> 32));
+}
+
+__device__ __forceinline__ void load_scale_atoms(const uint64_t* rows, int n_rows, uint8_t* atom0,
+                                                 uint8_t* atom1, int lane) {
+    uint64_t w[4];
+    fetch_scales(rows, n_rows, lane, w);
+    store_scale_atoms(w, atom0, atom1, lane);
 }
 
 __device__ __forceinline__ uint64_t atom_desc(const void* atom) {
@@ -200,12 +223,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
         mbar_init(smem_u32(&sm.bar_s_full[0]), 1);
         mbar_init(smem_u32(&sm.bar_s_full[1]), 1);
-        mbar_init(smem_u32(&sm.bar_p_ready), SOFTMAX_WARPS * 32);
+        mbar_init(smem_u32(&sm.bar_p_ready[0]), SOFTMAX_WARPS * 32);
+        mbar_init(smem_u32(&sm.bar_p_ready[1]), SOFTMAX_WARPS * 32);
         mbar_init(smem_u32(&sm.bar_o_done), 1);
+        mbar_init(smem_u32(&sm.bar_o_final), 1);
         mbar_init(smem_u32(&sm.bar_final), 1);
         for (int q = 0; q < 4; ++q) {
-            mbar_init(smem_u32(&sm.bar_pair[q][0]), 64);
-            mbar_init(smem_u32(&sm.bar_pair[q][1]), 64);
+            mbar_init(smem_u32(&sm.bar_group[q][0]), 32 * COL_GROUPS);
+            mbar_init(smem_u32(&sm.bar_group[q][1]), 32 * COL_GROUPS);
         }
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -241,6 +266,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             tma_load_3d(smem_u32(sm.qc), &tm_qc, 0, q0, bh, qf);
         }
         int issued = 0;
+        uint64_t ksc[4];  // the next tile's scales, fetched before its stage is free
+        fetch_scales(ks_head, N, lane, ksc);
         for (int j = 0; j < T; ++j) {
             const int s = j % STAGES;
             if (j >= STAGES) {
@@ -249,7 +276,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     break;
             }
             const int k0 = j * BN;
-            load_scale_atoms(ks_head + k0, N - k0, sm.ks_atom[s][0], sm.ks_atom[s][1], lane);
+            store_scale_atoms(ksc, sm.ks_atom[s][0], sm.ks_atom[s][1], lane);
+            if (j + 1 < T) fetch_scales(ks_head + k0 + BN, N - k0 - BN, lane, ksc);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -280,12 +308,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             __syncwarp();
         }
         auto pv_step = [&](int i) -> bool {
-            if (!warp_wait(smem_u32(&sm.bar_p_ready), i & 1, abort_flag, p.status, limit)) return false;
+            if (!warp_wait(smem_u32(&sm.bar_p_ready[i & 1]), (i >> 1) & 1, abort_flag, p.status, limit))
+                return false;
             if (lane == 0) {
                 tc_fence_after();
                 issue_pv(tmem, TM_S0 + 128u * (i & 1), sm.v[i % STAGES], i > 0);
                 tc_commit(smem_u32(&sm.bar_kv_empty[i % STAGES]));
                 tc_commit(smem_u32(&sm.bar_o_done));
+                if (i == T - 1) tc_commit(smem_u32(&sm.bar_o_final));
             }
             __syncwarp();
             return true;
@@ -320,8 +350,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ softmax warps --
-        const int quad = warp & 3;   // TMEM sub-partition: rows 32*quad ..
-        const int half = warp >> 2;  // keys 64*half .. 64*half+63 of each tile
+        const int quad = warp & 3;  // TMEM sub-partition: rows 32*quad ..
+        const int grp = warp >> 2;  // score columns CW*grp .. CW*grp+CW-1 of each tile
         const int row = 32 * quad + lane;
         const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
         float gq = 1.0f, gk = 1.0f;
@@ -344,38 +374,44 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t sr[2][32];
-            tmem_ld32(s_addr + 64u * half, sr[0]);
-            tmem_ld32(s_addr + 64u * half + 32u, sr[1]);
-            tmem_wait_ld();
-            const int nvalid = N - j * BN - 64 * half;
-            if (nvalid < 64) {
+            uint32_t sr[CW32][32];
 #pragma unroll
-                for (int q = 0; q < 2; ++q)
+            for (int q = 0; q < CW32; ++q) tmem_ld32(s_addr + (uint32_t)(CW * grp + 32 * q), sr[q]);
+            tmem_wait_ld();
+            const int nvalid = N - j * BN - CW * grp;
+            if (nvalid < CW) {
+#pragma unroll
+                for (int q = 0; q < CW32; ++q)
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (32 * q + i >= nvalid) sr[q][i] = __float_as_uint(-INFINITY);
             }
-            // partial row max of this half: a tree of three-input maxima
-            float a[8];
+            // partial row max of this warp's columns: a tree of three-input maxima
+            float a[CW / 8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < CW / 8; ++k) {
                 const uint32_t* v = &sr[k >> 2][(k & 3) * 8];
                 a[k] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
                              fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
                              fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
             }
-            const float pmax = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-            // exchange with the other half of the row (all S reads of the tile are done after this)
-            sm.red_max[b][half][row] = pmax;
+            float pmax = a[0];
+#pragma unroll
+            for (int k = 1; k < CW / 8; ++k) pmax = fmaxf(pmax, a[k]);
+            // exchange with the other column groups of the same rows (after this
+            // every S read of the tile is done, so P may overwrite S)
+            sm.red_max[b][grp][row] = pmax;
             tc_fence_before();
-            mbar_arrive(smem_u32(&sm.bar_pair[quad][b]));
-            if (!warp_wait(smem_u32(&sm.bar_pair[quad][b]), (j >> 1) & 1, abort_flag, p.status, limit)) {
+            mbar_arrive(smem_u32(&sm.bar_group[quad][b]));
+            if (!warp_wait(smem_u32(&sm.bar_group[quad][b]), (j >> 1) & 1, abort_flag, p.status, limit)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const float mx = fmaxf(pmax, sm.red_max[b][half ^ 1][row]) * c;
+            float tmax = sm.red_max[b][0][row];
+#pragma unroll
+            for (int g = 1; g < COL_GROUPS; ++g) tmax = fmaxf(tmax, sm.red_max[b][g][row]);
+            const float mx = tmax * c;
             float alpha = 1.0f;
             bool rescale = false;
             if (mx > m_run + 8.0f) {
@@ -387,9 +423,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 for (int k = 0; k < 4; ++k) lacc[k] = __fmul2_rn(lacc[k], a2);
             }
             const float2 negm = make_float2(-m_run, -m_run);
-            uint32_t pk[32];
+            uint32_t pk[CW / 2];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
+            for (int k = 0; k < CW / 2; ++k) {
                 const float2 s2 = make_float2(__uint_as_float(sr[k >> 4][(2 * k) & 31]),
                                               __uint_as_float(sr[k >> 4][(2 * k + 1) & 31]));
                 const float2 x = __ffma2_rn(s2, c2, negm);
@@ -402,61 +438,68 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 lacc[k & 3] = __fadd2_rn(lacc[k & 3], pv);
                 pk[k] = pack_bf16x2(pv.x, pv.y);
             }
-            // P (bf16 pairs) over this half's 32 columns of the S buffer
-            tmem_st32(s_addr + 32u * half, pk);
+            // P (bf16 pairs) over this warp's CW/2 columns of the S buffer
+            if constexpr (CW == 64) {
+                tmem_st32(s_addr + 32u * grp, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+            } else {
+                tmem_st16(s_addr + 16u * grp, pk);
+            }
             tmem_wait_st();
-            if (j >= 1) {
-                // O holds the sum up to tile j-1 once that tile's P.V is done
+            // tcgen05.ld/st are warp-collective: the whole warp takes this branch
+            // when any of its rows needs it (alpha is 1 elsewhere).  Only then
+            // does it wait for tile j-1's P.V: S(j) being ready means every
+            // earlier P.V has completed, so that is the only one in flight and
+            // the parity wait is unambiguous.
+            if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
                 if (!warp_wait(smem_u32(&sm.bar_o_done), (j - 1) & 1, abort_flag, p.status, limit)) {
                     ok = false;
                     break;
                 }
-                // tcgen05.ld/st are warp-collective: the whole warp takes this
-                // branch when any of its rows needs it (alpha is 1 elsewhere)
-                if (__any_sync(0xffffffffu, rescale)) {
-                    tc_fence_after();
-                    const uint32_t o_addr = tmem + lane_base + TM_O + 64u * half;
-                    const float2 a2 = make_float2(alpha, alpha);
+                tc_fence_after();
+                const uint32_t o_addr = tmem + lane_base + TM_O + (uint32_t)(CW * grp);
+                const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint32_t r[32];
-                        tmem_ld32(o_addr + 32u * q, r);
-                        tmem_wait_ld();
+                for (int q = 0; q < CW32; ++q) {
+                    uint32_t r[32];
+                    tmem_ld32(o_addr + 32u * q, r);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2);
-                            r[i] = __float_as_uint(o2.x);
-                            r[i + 1] = __float_as_uint(o2.y);
-                        }
-                        tmem_st32(o_addr + 32u * q, r);
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 o2 =
+                            __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2);
+                        r[i] = __float_as_uint(o2.x);
+                        r[i + 1] = __float_as_uint(o2.y);
                     }
-                    tmem_wait_st();
+                    tmem_st32(o_addr + 32u * q, r);
                 }
+                tmem_wait_st();
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&sm.bar_p_ready));
+            mbar_arrive(smem_u32(&sm.bar_p_ready[b]));
         }
         if (ok && T > 0) {
-            // total row sum from both halves (the pair barrier's next phase)
-            const float l_half = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) + (lacc[2].x + lacc[2].y) +
+            // total row sum over the column groups (the group barrier's next phase)
+            const float l_part = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) + (lacc[2].x + lacc[2].y) +
                                  (lacc[3].x + lacc[3].y);
-            sm.red_sum[half][row] = l_half;
-            mbar_arrive(smem_u32(&sm.bar_pair[quad][T & 1]));
-            ok = warp_wait(smem_u32(&sm.bar_pair[quad][T & 1]), (T >> 1) & 1, abort_flag, p.status, limit);
-            const float l = l_half + sm.red_sum[half ^ 1][row];
-            if (ok && warp_wait(smem_u32(&sm.bar_o_done), (T - 1) & 1, abort_flag, p.status, limit)) {
+            sm.red_sum[grp][row] = l_part;
+            mbar_arrive(smem_u32(&sm.bar_group[quad][T & 1]));
+            ok = warp_wait(smem_u32(&sm.bar_group[quad][T & 1]), (T >> 1) & 1, abort_flag, p.status, limit);
+            float l = sm.red_sum[0][row];
+#pragma unroll
+            for (int g = 1; g < COL_GROUPS; ++g) l += sm.red_sum[g][row];
+            if (ok && warp_wait(smem_u32(&sm.bar_o_final), 0, abort_flag, p.status, limit)) {
                 tc_fence_after();
                 const float inv_l = 1.0f / l;
-                const uint32_t o_addr = tmem + lane_base + TM_O + 64u * half;
+                const uint32_t o_addr = tmem + lane_base + TM_O + (uint32_t)(CW * grp);
                 const int n = q0 + row;
                 const size_t orow = (size_t)bh * N + n;
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < CW32; ++q) {
                     uint32_t r[32];
                     tmem_ld32(o_addr + 32u * q, r);
                     tmem_wait_ld();
                     if (n < N) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + 64 * half + 32 * q);
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + CW * grp + 32 * q);
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             uint32_t w[4];
@@ -469,7 +512,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                         }
                     }
                 }
-                if (p.lse && n < N && half == 0) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
+                if (p.lse && n < N && grp == 0) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
             }
         }
     }
