@@ -4,28 +4,31 @@
 // Method: FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention":
 // queries and keys are quantised for an NVFP4 attention kernel; P and V stay
 // in BF16.  This kernel is written for sm_100a:
-//   * one CTA per (head, 128-query tile); 4 * COL_GROUPS softmax warps plus
-//     two more:
-//       softmax    softmax, O correction and epilogue; query row r is TMEM
-//                  lane r and is shared by the COL_GROUPS warps w with
-//                  w % 4 == r / 32, each owning 128 / COL_GROUPS key columns
-//                  of every tile; they exchange partial row maxima through
-//                  shared memory every tile;
-//       producer   scale-factor atoms (plain loads) and TMA copies of Q
-//                  once, then K codes and V tiles of 128 keys into a
-//                  STAGES-deep shared-memory ring;
-//       MMA        TMEM owner and MMA issuer: stages the scale factors into
-//                  TMEM (tcgen05.cp) and issues S = Q K^T with
-//                  tcgen05.mma kind::mxf4nvf4 (block16 scales) and
-//                  O += P V with tcgen05.mma kind::f16 (P read from TMEM);
-//   * TMEM (512 columns): S double buffer [0,128) [128,256) fp32, O [256,384),
-//     Q scale factors [384,392), K scale factors 2 x 8 columns from 392; P is
-//     written as bf16 pairs over the first 64 columns of its S buffer;
-//   * online softmax in the log2 domain with a lazy rescale: the running max
-//     only moves when a tile's max exceeds it by more than 8 (so p <= 256),
-//     and O is rescaled in TMEM only then; exponentials are split between
-//     the MUFU unit and a polynomial on the FMA pipe, with packed fp32x2
-//     arithmetic for the scale, the polynomial and the row sums.
+//   * one CTA per (head, 256 queries) = two 128-row query tiles that share
+//     every K/V tile loaded into shared memory; 320 threads:
+//       warps 0-3  softmax of query tile 0, warps 4-7 softmax of tile 1 (one
+//                  warp per TMEM sub-partition, one query row per thread);
+//       warp 8     producer: scale-factor atoms (plain loads) and TMA copies
+//                  of both Q tiles once, then K codes and V of 112 keys per
+//                  stage into a STAGES-deep shared-memory ring;
+//       warp 9     TMEM owner and MMA issuer: stages scale factors into TMEM
+//                  (tcgen05.cp), S_i = Q_i K^T with tcgen05.mma
+//                  kind::mxf4nvf4 (block16 UE4M3 scales) into TMEM, and
+//                  O_i += P_i V with tcgen05.mma kind::f16 from shared memory;
+//   * P_i goes to shared memory (K-major, 32-byte swizzle, one 4 KB panel per
+//     16 keys), not back into TMEM, so S_i is free as soon as its softmax
+//     warps have loaded it: S_i of the next stage is computed while they
+//     still work on this one, and each softmax warp group moves from stage to
+//     stage without waiting for the tensor cores;
+//   * TMEM (512 columns): S_0 [0,112), S_1 [112,224) fp32, O_0 [224,352),
+//     O_1 [352,480), the two Q tiles' scale factors [480,496) and two slots
+//     of K scale factors [496,512).  112 keys per stage is what lets four
+//     accumulators and the scale factors fit the 512 columns together;
+//   * online softmax in the log2 domain with a lazy running max: the max
+//     only moves when a stage's max exceeds it by more than 8 (so p <= 256),
+//     and only then is O_i rescaled in TMEM, after the previous P_i V has
+//     completed.  Exponentials are split between MUFU ex2 and a polynomial on
+//     the FMA pipe, with packed fp32x2 arithmetic.
 // Every wait is bounded; a wait that runs out raises FP4ATTN_ERR_TIMEOUT in
 // the status word and the CTA winds down (waiting for its own copies and MMAs)
 // instead of hanging.
@@ -38,65 +41,70 @@ namespace fp4attn {
 
 namespace {
 
-constexpr int BM = 128;  // query rows per CTA
-constexpr int BN = 128;  // keys per tile
+constexpr int BM = 128;  // query rows per tile
+constexpr int QT = 2;    // query tiles per CTA
+constexpr int BN = 112;  // keys per K/V stage
 constexpr int STAGES = 4;
-// Softmax warps come in COL_GROUPS groups of four (one warp per TMEM
-// sub-partition); each warp owns CW of the 128 score columns of its 32 rows.
-#ifndef FP4ATTN_COL_GROUPS
-#define FP4ATTN_COL_GROUPS 2
-#endif
+constexpr int SOFTMAX_WARPS = 4 * QT;
+// Warpgroups 0 and 1 are the softmax warps, warpgroup 2 holds the producer and
+// the MMA warp (its last two warps only take part in the register split).
+constexpr int FWD_THREADS = 32 * (SOFTMAX_WARPS + 4);
+constexpr int WARP_PRODUCER = SOFTMAX_WARPS;
+constexpr int WARP_MMA = SOFTMAX_WARPS + 1;
+// Register split: three warps share each SM sub-partition's 16384 registers,
+// so the launch gets 168 per thread; the producer/MMA warpgroup gives most of
+// its share to the softmax warpgroups (2 x 128 x 232 + 128 x 40 = 384 x 168).
+constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 224, SUPPORT_REGS = 56;
+static_assert(2 * 128 * SOFTMAX_REGS + 128 * SUPPORT_REGS <= FWD_THREADS * LAUNCH_REGS, "register split");
+static_assert((2 * SOFTMAX_REGS + SUPPORT_REGS) * 32 <= 16384, "registers of one SM sub-partition");
 // Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
 // and the rest to MUFU ex2 (MUFU issues 16 per clock per SM).
 #ifndef FP4ATTN_POLY_PAIRS
 #define FP4ATTN_POLY_PAIRS 3
 #endif
-constexpr int COL_GROUPS = FP4ATTN_COL_GROUPS;
-static_assert(COL_GROUPS == 2 || COL_GROUPS == 4, "2 or 4 column groups");
-constexpr int CW = 128 / COL_GROUPS;  // score columns per softmax warp
-constexpr int CW32 = CW / 32;         // 32-column TMEM loads per tile
-constexpr int SOFTMAX_WARPS = 4 * COL_GROUPS;
-constexpr int FWD_THREADS = 32 * (SOFTMAX_WARPS + 2);
-constexpr int WARP_PRODUCER = SOFTMAX_WARPS;
-constexpr int WARP_MMA = SOFTMAX_WARPS + 1;
 constexpr int POLY_PAIRS_PER_8 = FP4ATTN_POLY_PAIRS;
 
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0;
-constexpr uint32_t TM_O = 256;
-constexpr uint32_t TM_SFQ = 384;
-constexpr uint32_t TM_SFK = 392;
+__host__ __device__ constexpr uint32_t tm_s(int i) { return (uint32_t)(BN * i); }
+__host__ __device__ constexpr uint32_t tm_o(int i) { return (uint32_t)(2 * BN + 128 * i); }
+__host__ __device__ constexpr uint32_t tm_sfq(int i) { return (uint32_t)(2 * BN + 256 + 8 * i); }
+__host__ __device__ constexpr uint32_t tm_sfk(int slot) { return (uint32_t)(2 * BN + 256 + 16 + 8 * slot); }
+static_assert(tm_sfk(1) + 8 == TMEM_COLS, "TMEM budget");
 
-constexpr uint32_t CODE_TILE_BYTES = 128 * 64;    // 128 rows x 128 E2M1 values
-constexpr uint32_t V_PANEL_BYTES = 128 * 64 * 2;  // 128 keys x 64 channels bf16
+constexpr uint32_t Q_TILE_BYTES = BM * 64;         // 128 rows x 128 E2M1 values
+constexpr uint32_t K_TILE_BYTES = BN * 64;         // 112 rows x 128 E2M1 values
+constexpr uint32_t V_PANEL_BYTES = BN * 64 * 2;    // 112 keys x 64 channels bf16
 constexpr uint32_t V_TILE_BYTES = 2 * V_PANEL_BYTES;
+static_assert(K_TILE_BYTES % 1024 == 0 && V_PANEL_BYTES % 1024 == 0, "swizzle atoms stay 1 KB aligned");
+// P in shared memory: one panel per 16 keys, 128 rows x 32 bytes (16 bf16),
+// K-major with the 32-byte swizzle (the two 16-byte halves of a row swap
+// places in rows 4-7 of every 8-row group); 8-row groups 256 B apart.
+constexpr uint32_t P_PANEL_BYTES = BM * 32;
+constexpr uint32_t P_TILE_BYTES = (BN / 16) * P_PANEL_BYTES;
 
 // Instruction descriptors.
-//  S: kind::mxf4nvf4, A = B = E2M1 (1), UE4M3 scales, K-major, N = 128, M = 128.
-constexpr uint32_t IDESC_QK = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                              ((uint32_t)(BM >> 4) << 24);
-//  O: kind::f16, fp32 accumulate (1 << 4), A = B = BF16, A K-major (TMEM),
+//  S: kind::mxf4nvf4, A = B = E2M1 (1), UE4M3 scales, K-major, M = 128, N = n keys.
+__host__ __device__ constexpr uint32_t idesc_qk(int n) { return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24); }
+//  O: kind::f16, fp32 accumulate (1 << 4), A = B = BF16, A = P K-major,
 //     B = V MN-major (1 << 16), N = 128 channels, M = 128.
 constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                               ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 struct __align__(1024) FwdSmem {
-    uint8_t v[STAGES][V_TILE_BYTES];      // two 64-channel panels, 128B swizzle
-    uint8_t kc[STAGES][CODE_TILE_BYTES];  // 64B swizzle
-    uint8_t qc[CODE_TILE_BYTES];          // 64B swizzle
-    uint8_t ks_atom[STAGES][2][512];      // scale-factor atoms for tcgen05.cp
-    uint8_t qs_atom[2][512];
+    uint8_t v[STAGES][V_TILE_BYTES];   // two 64-channel panels, 128B swizzle
+    uint8_t kc[STAGES][K_TILE_BYTES];  // 64B swizzle
+    uint8_t qc[QT][Q_TILE_BYTES];      // 64B swizzle
+    uint8_t pb[QT][P_TILE_BYTES];      // P_i, 32B swizzle
+    uint8_t ks_atom[STAGES][2][512];   // scale-factor atoms for tcgen05.cp
+    uint8_t qs_atom[QT][2][512];
     uint64_t bar_q_full;
     uint64_t bar_kv_full[STAGES];
     uint64_t bar_kv_empty[STAGES];
-    uint64_t bar_s_full[2];
-    uint64_t bar_p_ready[2];      // P of tiles with this parity is in TMEM
-    uint64_t bar_o_done;          // O holds the P.V of every tile up to the last commit
-    uint64_t bar_o_final;         // the last tile's P.V is done
-    uint64_t bar_final;
-    uint64_t bar_group[4][2];              // per sub-partition, per tile parity: all partial maxima are in
-    float red_max[2][COL_GROUPS][128];     // [tile parity][column group][row] partial row maxima
-    float red_sum[COL_GROUPS][128];        // [column group][row] partial row sums, at the end
+    uint64_t bar_s_full[QT];   // S_i of the next stage is in TMEM
+    uint64_t bar_s_free[QT];   // the softmax warps of tile i have loaded S_i into registers
+    uint64_t bar_p_full[QT];   // P_i of the stage is in shared memory (O_i rescaled if needed)
+    uint64_t bar_pv_done[QT];  // O_i += P_i V of the stage has completed (P_i buffer free)
+    uint64_t bar_final;        // every MMA and copy of the CTA has completed
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -105,7 +113,7 @@ struct FwdParams {
     const uint64_t* q_scales;  // one uint64 (8 UE4M3 bytes) per row
     const uint64_t* k_scales;
     int N;
-    int n_kt;
+    int n_kt;          // K/V stages of BN keys
     float scale_log2;  // softmax_scale * log2(e)
     const float* gq;
     const float* gk;
@@ -136,13 +144,14 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
     return mbar_wait(bar, parity, &dummy_abort, nullptr, kDrainLimitNs);
 }
 
-// Scales of 128 rows (row-major, one uint64 = 8 UE4M3 bytes per row) -> two
-// 512-byte atoms (channels 0-63 and 64-127).  Atom line r (16 bytes) holds,
-// for rows r, r+32, r+64, r+96, the four scales of that 64-channel chunk;
-// tcgen05.cp 32x128b.warpx4 then puts line r in TMEM lane r of every
-// sub-partition.  One full warp, lane = line; rows at or beyond n_rows read
-// as zero.  Plain 8-byte loads: a row's scales start at any multiple of 8
-// bytes, which a bulk tensor copy could not address.
+// Scales of up to 128 rows (row-major, one uint64 = 8 UE4M3 bytes per row) ->
+// two 512-byte atoms (channels 0-63 and 64-127).  Atom line r (16 bytes)
+// holds, for rows r, r+32, r+64, r+96, the four scales of that 64-channel
+// chunk; tcgen05.cp 32x128b.warpx4 then puts line r in TMEM lane r of every
+// sub-partition, so rows 32c.. sit in column c of the chunk's four columns.
+// One full warp, lane = line; rows at or beyond n_rows read as zero.  Plain
+// 8-byte loads: a row's scales start at any multiple of 8 bytes, which a bulk
+// tensor copy could not address.
 __device__ __forceinline__ void fetch_scales(const uint64_t* rows, int n_rows, int lane, uint64_t (&w)[4]) {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -176,29 +185,56 @@ __device__ __forceinline__ uint64_t codes_desc(const uint8_t* tile, int kchunk) 
     return smem_desc(smem_u32(tile) + 32u * kchunk, 16, 512, LAYOUT_SW64);
 }
 
-__device__ __forceinline__ uint64_t v_desc(const uint8_t* tile, int kstep) {
-    // MN-major 128B swizzle: 64-channel panels 16 KB apart (leading byte
-    // offset), 8-key groups 1 KB apart (stride byte offset); one MMA covers
-    // 16 keys = 2 KB of each panel.
-    return smem_desc(smem_u32(tile) + 2048u * kstep, V_PANEL_BYTES, 1024, LAYOUT_SW128);
+__device__ __forceinline__ uint64_t v_desc(const uint8_t* tile, int kstep, uint32_t panel_bytes) {
+    // MN-major 128B swizzle: the two 64-channel panels panel_bytes apart
+    // (leading byte offset), 8-key groups 1 KB apart (stride byte offset);
+    // one MMA covers 16 keys = 2 KB of each panel.
+    return smem_desc(smem_u32(tile) + 2048u * kstep, panel_bytes, 1024, LAYOUT_SW128);
 }
 
-// Issue S = Q K^T for one key tile (two K=64 block-scaled MMAs).
-__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t s_col, const uint8_t* qc,
-                                         const uint8_t* kc, uint32_t sfk_col) {
+__device__ __forceinline__ uint64_t p_desc(const uint8_t* p_tile, int kstep) {
+    // K-major 32B swizzle: one panel of 128 rows x 32 bytes per 16 keys,
+    // 8-row groups 256 B apart (stride byte offset); the leading byte offset
+    // is unused because one MMA's K extent is the swizzle width.
+    return smem_desc(smem_u32(p_tile) + P_PANEL_BYTES * kstep, 16, 256, LAYOUT_SW32);
+}
+
+// Row `row` of P (NP panels of 16 keys; pk = 8 NP bf16 pairs, key order) into
+// the 32B-swizzled layout p_desc reads.  A warp's 32 rows hit all 32 banks
+// once per 8 lanes, so each 16-byte store takes the minimum four wavefronts.
+template <int NP>
+__device__ __forceinline__ void store_p_row(uint8_t* p_tile, int row, const uint32_t* pk) {
+    const uint32_t sw = (uint32_t)(row >> 2) & 1u;
+    uint8_t* base = p_tile + 32 * row;
 #pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-        mma_mxf4nvf4(tmem + s_col, codes_desc(qc, kk), codes_desc(kc, kk), IDESC_QK,
-                     tmem + TM_SFQ + 4u * kk, tmem + sfk_col + 4u * kk, kk > 0 ? 1u : 0u);
+    for (int ks = 0; ks < NP; ++ks) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t* w = pk + 8 * ks + 4 * h;
+            *reinterpret_cast<uint4*>(base + P_PANEL_BYTES * ks + 16u * ((uint32_t)h ^ sw)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
 }
 
-// Issue O (+)= P V for one key tile (eight K=16 BF16 MMAs, P from TMEM).
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t p_col, const uint8_t* v,
-                                         bool accumulate_first) {
+// S = Q K^T over all 128 channels for one query tile and n keys: two K=64
+// block-scaled MMAs, scale factors of Q at sfq_col, of K at sfk_col.
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t s_col, const uint8_t* qc, const uint8_t* kc,
+                                         uint32_t sfq_col, uint32_t sfk_col, uint32_t idesc) {
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-        mma_bf16_ts(tmem + TM_O, tmem + p_col + 8u * ks, v_desc(v, ks), IDESC_PV,
+    for (int kk = 0; kk < 2; ++kk) {
+        mma_mxf4nvf4(tmem + s_col, codes_desc(qc, kk), codes_desc(kc, kk), idesc, tmem + sfq_col + 4u * kk,
+                     tmem + sfk_col + 4u * kk, kk > 0 ? 1u : 0u);
+    }
+}
+
+// O (+)= P V over NK keys (NK/16 K=16 BF16 MMAs, P from shared memory).
+template <int NK>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t o_col, const uint8_t* p_tile, const uint8_t* v,
+                                         uint32_t v_panel_bytes, bool accumulate_first) {
+#pragma unroll
+    for (int ks = 0; ks < NK / 16; ++ks) {
+        mma_bf16_ss(tmem + o_col, p_desc(p_tile, ks), v_desc(v, ks, v_panel_bytes), IDESC_PV,
                     (accumulate_first || ks > 0) ? 1u : 0u);
     }
 }
@@ -211,7 +247,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
-    const int q0 = blockIdx.x * BM;
+    const int q0 = blockIdx.x * (QT * BM);
     const int T = p.n_kt;
     const int N = p.N;
 
@@ -221,17 +257,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             mbar_init(smem_u32(&sm.bar_kv_full[s]), 1);
             mbar_init(smem_u32(&sm.bar_kv_empty[s]), 1);
         }
-        mbar_init(smem_u32(&sm.bar_s_full[0]), 1);
-        mbar_init(smem_u32(&sm.bar_s_full[1]), 1);
-        mbar_init(smem_u32(&sm.bar_p_ready[0]), SOFTMAX_WARPS * 32);
-        mbar_init(smem_u32(&sm.bar_p_ready[1]), SOFTMAX_WARPS * 32);
-        mbar_init(smem_u32(&sm.bar_o_done), 1);
-        mbar_init(smem_u32(&sm.bar_o_final), 1);
-        mbar_init(smem_u32(&sm.bar_final), 1);
-        for (int q = 0; q < 4; ++q) {
-            mbar_init(smem_u32(&sm.bar_group[q][0]), 32 * COL_GROUPS);
-            mbar_init(smem_u32(&sm.bar_group[q][1]), 32 * COL_GROUPS);
+        for (int i = 0; i < QT; ++i) {
+            mbar_init(smem_u32(&sm.bar_s_full[i]), 1);
+            mbar_init(smem_u32(&sm.bar_s_free[i]), 128);
+            mbar_init(smem_u32(&sm.bar_p_full[i]), 128);
+            mbar_init(smem_u32(&sm.bar_pv_done[i]), 1);
         }
+        mbar_init(smem_u32(&sm.bar_final), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -250,24 +282,32 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     const uint32_t tmem = sm.tmem_base;
     volatile int* abort_flag = &sm.abort_flag;
     const uint64_t limit = p.limit_ns;
-
+    if (warp >= SOFTMAX_WARPS) {
+    setmaxnreg_dec<SUPPORT_REGS>();
     if (warp == WARP_PRODUCER) {
         // ------------------------------------------------------ producer --
         // All 32 lanes stage the scale atoms; lane 0 arms the barrier and
-        // issues the bulk tensor copies after the atoms are written.
+        // issues the bulk tensor copies after the atoms are written.  A query
+        // tile that lies past N is copied all the same (the copy fills zeros)
+        // and its rows are never stored.
         const uint64_t* qs_head = p.q_scales + (size_t)bh * N;
         const uint64_t* ks_head = p.k_scales + (size_t)bh * N;
         const uint32_t qf = smem_u32(&sm.bar_q_full);
-        load_scale_atoms(qs_head + q0, N - q0, sm.qs_atom[0], sm.qs_atom[1], lane);
+#pragma unroll
+        for (int i = 0; i < QT; ++i) {
+            const int r0 = q0 + BM * i;
+            load_scale_atoms(qs_head + (r0 < N ? r0 : 0), N - r0, sm.qs_atom[i][0], sm.qs_atom[i][1], lane);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive_expect_tx(qf, CODE_TILE_BYTES);
-            tma_load_3d(smem_u32(sm.qc), &tm_qc, 0, q0, bh, qf);
+            mbar_arrive_expect_tx(qf, QT * Q_TILE_BYTES);
+#pragma unroll
+            for (int i = 0; i < QT; ++i) tma_load_3d(smem_u32(sm.qc[i]), &tm_qc, 0, q0 + BM * i, bh, qf);
         }
         int issued = 0;
-        uint64_t ksc[4];  // the next tile's scales, fetched before its stage is free
-        fetch_scales(ks_head, N, lane, ksc);
+        uint64_t ksc[4];  // the next stage's scales, fetched before its buffer is free
+        fetch_scales(ks_head, N < BN ? N : BN, lane, ksc);
         for (int j = 0; j < T; ++j) {
             const int s = j % STAGES;
             if (j >= STAGES) {
@@ -277,12 +317,15 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             }
             const int k0 = j * BN;
             store_scale_atoms(ksc, sm.ks_atom[s][0], sm.ks_atom[s][1], lane);
-            if (j + 1 < T) fetch_scales(ks_head + k0 + BN, N - k0 - BN, lane, ksc);
+            if (j + 1 < T) {
+                const int rest = N - k0 - BN;
+                fetch_scales(ks_head + k0 + BN, rest < BN ? rest : BN, lane, ksc);
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 const uint32_t full = smem_u32(&sm.bar_kv_full[s]);
-                mbar_arrive_expect_tx(full, CODE_TILE_BYTES + V_TILE_BYTES);
+                mbar_arrive_expect_tx(full, K_TILE_BYTES + V_TILE_BYTES);
                 tma_load_3d(smem_u32(sm.kc[s]), &tm_kc, 0, k0, bh, full);
                 tma_load_3d(smem_u32(sm.v[s]), &tm_v, 0, k0, bh, full);
                 tma_load_3d(smem_u32(sm.v[s]) + V_PANEL_BYTES, &tm_v, 64, k0, bh, full);
@@ -298,62 +341,126 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         // ----------------------------------------------------------- MMA --
-        bool ok = warp_wait(smem_u32(&sm.bar_q_full), 0, abort_flag, p.status, limit);
-        if (ok) {
-            if (lane == 0) {
-                tc_fence_after();
-                tmem_cp_32x128b_x4(tmem + TM_SFQ, atom_desc(sm.qs_atom[0]));
-                tmem_cp_32x128b_x4(tmem + TM_SFQ + 4, atom_desc(sm.qs_atom[1]));
-            }
-            __syncwarp();
-        }
-        auto pv_step = [&](int i) -> bool {
-            if (!warp_wait(smem_u32(&sm.bar_p_ready[i & 1]), (i >> 1) & 1, abort_flag, p.status, limit))
-                return false;
-            if (lane == 0) {
-                tc_fence_after();
-                issue_pv(tmem, TM_S0 + 128u * (i & 1), sm.v[i % STAGES], i > 0);
-                tc_commit(smem_u32(&sm.bar_kv_empty[i % STAGES]));
-                tc_commit(smem_u32(&sm.bar_o_done));
-                if (i == T - 1) tc_commit(smem_u32(&sm.bar_o_final));
-            }
-            __syncwarp();
-            return true;
+        // Issue order: S_0(0) S_1(0) S_0(1) S_1(1), then per stage j
+        //   O_0 += P_0(j) V_j,  S_0(j+2),  O_1 += P_1(j) V_j,  S_1(j+2).
+        // S_i(j+2) waits until the softmax warps have loaded S_i(j+1), and
+        // O_i += P_i(j) V_j until P_i(j) is in shared memory; the softmax
+        // warps only ever wait for work issued before, so nothing can wait
+        // in a circle.  A K scale-factor slot is refilled for stage j+2 once
+        // S_0(j+1) has been loaded: S_0(j+1) was issued after the last reader
+        // of the slot (S_1(j)), and tcgen05 operations of one thread complete
+        // in order.
+        //
+        // This warp is on the critical path of both tiles, so it keeps its
+        // instruction stream short: every shared-memory descriptor is a base
+        // computed once plus a constant (the address field of a descriptor
+        // is the byte address / 16 and never carries into the next field,
+        // shared memory being below 256 KB), the descriptors live in
+        // warp-uniform registers and one elected lane issues, and its waits
+        // poll instead of suspending.
+        const bool leader = elect_one_sync();
+        const uint64_t qd = codes_desc(sm.qc[0], 0);      // tile i: + i*Q_TILE/16, chunk kk: + 2 kk
+        const uint64_t kd0 = codes_desc(sm.kc[0], 0);     // stage st: + st*K_TILE/16
+        const uint64_t vd0 = v_desc(sm.v[0], 0, V_PANEL_BYTES);  // stage st: + st*V_TILE/16, kstep: + 128
+        const uint64_t pd0 = p_desc(sm.pb[0], 0);         // tile i: + i*P_TILE/16, kstep: + P_PANEL/16
+        const uint64_t kad0 = atom_desc(sm.ks_atom[0][0]);  // stage st: + 64 st, half h: + 32 h
+        constexpr uint64_t QD_TILE = Q_TILE_BYTES >> 4, KD_STAGE = K_TILE_BYTES >> 4,
+                           VD_STAGE = V_TILE_BYTES >> 4, PD_TILE = P_TILE_BYTES >> 4,
+                           PD_STEP = P_PANEL_BYTES >> 4, AD_STAGE = (2 * 512) >> 4;
+        constexpr uint32_t IDESC_S = idesc_qk(BN);
+        auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, p.status, limit));
         };
-        for (int j = 0; ok && j < T; ++j) {
-            const int s = j % STAGES;
-            const int b = j & 1;
-            if (!warp_wait(smem_u32(&sm.bar_kv_full[s]), (j / STAGES) & 1, abort_flag, p.status, limit)) {
-                ok = false;
-                break;
+        // S_i(j): for i == 0 also stage the K scale factors of stage j
+        auto qk = [&](int i, int j) {
+            const int st = j % STAGES;
+            const uint32_t sfk = tm_sfk(j & 1);
+            const uint64_t kd = kd0 + KD_STAGE * st;
+            if (i == 0) {
+                const uint64_t kad = kad0 + AD_STAGE * st;
+                tmem_cp_32x128b_x4(tmem + sfk, kad);
+                tmem_cp_32x128b_x4(tmem + sfk + 4, kad + 32);
             }
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t sfk = TM_SFK + 8u * b;
-                tmem_cp_32x128b_x4(tmem + sfk, atom_desc(sm.ks_atom[s][0]));
-                tmem_cp_32x128b_x4(tmem + sfk + 4, atom_desc(sm.ks_atom[s][1]));
-                issue_qk(tmem, TM_S0 + 128u * b, sm.qc, sm.kc[s], sfk);
-                tc_commit(smem_u32(&sm.bar_s_full[b]));
-            }
-            __syncwarp();
-            if (j >= 1 && !pv_step(j - 1)) {
-                ok = false;
-                break;
+            mma_mxf4nvf4(tmem + tm_s(i), qd + QD_TILE * i, kd, IDESC_S, tmem + tm_sfq(i), tmem + sfk, 0u);
+            mma_mxf4nvf4(tmem + tm_s(i), qd + QD_TILE * i + 2, kd + 2, IDESC_S, tmem + tm_sfq(i) + 4,
+                         tmem + sfk + 4, 1u);
+            tc_commit(smem_u32(&sm.bar_s_full[i]));
+        };
+        auto pv = [&](int i, int j) {
+            const uint64_t vd = vd0 + VD_STAGE * (j % STAGES);
+            const uint64_t pd = pd0 + PD_TILE * i;
+#pragma unroll
+            for (int ks = 0; ks < BN / 16; ++ks)
+                mma_bf16_ss(tmem + tm_o(i), pd + PD_STEP * ks, vd + 128u * ks, IDESC_PV,
+                            (ks > 0 || j > 0) ? 1u : 0u);
+            tc_commit(smem_u32(&sm.bar_pv_done[i]));
+        };
+        bool ok = wait(smem_u32(&sm.bar_q_full), 0);
+        if (ok && leader) {
+            tc_fence_after();
+            const uint64_t qad = atom_desc(sm.qs_atom[0][0]);  // tile i: + 64 i, half h: + 32 h
+#pragma unroll
+            for (int i = 0; i < QT; ++i) {
+                tmem_cp_32x128b_x4(tmem + tm_sfq(i), qad + AD_STAGE * i);
+                tmem_cp_32x128b_x4(tmem + tm_sfq(i) + 4, qad + AD_STAGE * i + 32);
             }
         }
-        if (ok && T > 0) pv_step(T - 1);
+        __syncwarp();
+        // S of the first two stages
+        for (int j = 0; ok && j < 2 && j < T; ++j) {
+            ok = wait(smem_u32(&sm.bar_kv_full[j]), 0);
+            for (int i = 0; ok && i < QT; ++i) {
+                if (j == 1) ok = wait(smem_u32(&sm.bar_s_free[i]), 0);
+                if (ok && leader) {
+                    tc_fence_after();
+                    qk(i, j);
+                }
+                __syncwarp();
+            }
+        }
+        for (int j = 0; ok && j < T; ++j) {
+            const int jn = j + 2;  // stage whose S is computed next
+            for (int i = 0; i < QT; ++i) {
+                if (!wait(smem_u32(&sm.bar_p_full[i]), j & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (leader) {
+                    tc_fence_after();
+                    pv(i, j);
+                    if (i == QT - 1) tc_commit(smem_u32(&sm.bar_kv_empty[j % STAGES]));
+                }
+                __syncwarp();
+                if (jn < T) {
+                    if (!wait(smem_u32(&sm.bar_s_free[i]), (jn - 1) & 1) ||
+                        (i == 0 && !wait(smem_u32(&sm.bar_kv_full[jn % STAGES]), (jn / STAGES) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) {
+                        tc_fence_after();
+                        qk(i, jn);
+                    }
+                    __syncwarp();
+                }
+            }
+        }
         // every MMA and copy this warp issued must finish before TMEM is freed
-        if (lane == 0) {
+        if (leader) {
             tc_commit(smem_u32(&sm.bar_final));
             drain_wait(smem_u32(&sm.bar_final), 0);
         }
         __syncwarp();
+    }
     } else {
+        setmaxnreg_inc<SOFTMAX_REGS>();
         // ------------------------------------------------ softmax warps --
         const int quad = warp & 3;  // TMEM sub-partition: rows 32*quad ..
-        const int grp = warp >> 2;  // score columns CW*grp .. CW*grp+CW-1 of each tile
+        const int qt = warp >> 2;   // query tile of this warp group
         const int row = 32 * quad + lane;
         const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+        const uint32_t s_addr = tmem + lane_base + tm_s(qt);
+        const uint32_t o_addr = tmem + lane_base + tm_o(qt);
         float gq = 1.0f, gk = 1.0f;
         if (p.gq) gq = *p.gq;
         if (p.gk) gk = *p.gk;
@@ -362,72 +469,63 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
         const float c = p.scale_log2 * gq * gk;
         const float2 c2 = make_float2(c, c);
-        float m_run = -INFINITY;
+        float m_run = -INFINITY;  // running max (log2 domain) that P, O and the row sum are relative to
         float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
+        const uint32_t s_full = smem_u32(&sm.bar_s_full[qt]);
+        const uint32_t s_free = smem_u32(&sm.bar_s_free[qt]);
+        const uint32_t p_full = smem_u32(&sm.bar_p_full[qt]);
+        const uint32_t pv_done = smem_u32(&sm.bar_pv_done[qt]);
+        uint8_t* p_tile = sm.pb[qt];
         bool ok = true;
         for (int j = 0; j < T; ++j) {
-            const int b = j & 1;
-            const uint32_t s_addr = tmem + lane_base + TM_S0 + 128u * b;
-            if (!warp_wait(smem_u32(&sm.bar_s_full[b]), (j >> 1) & 1, abort_flag, p.status, limit)) {
+            if (!warp_wait(s_full, j & 1, abort_flag, p.status, limit)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t sr[CW32][32];
-#pragma unroll
-            for (int q = 0; q < CW32; ++q) tmem_ld32(s_addr + (uint32_t)(CW * grp + 32 * q), sr[q]);
+            uint32_t sr[BN];
+            tmem_ld32(s_addr, &sr[0]);
+            tmem_ld32(s_addr + 32u, &sr[32]);
+            tmem_ld32(s_addr + 64u, &sr[64]);
+            tmem_ld16(s_addr + 96u, &sr[96]);
             tmem_wait_ld();
-            const int nvalid = N - j * BN - CW * grp;
-            if (nvalid < CW) {
+            // S_i is in registers: the MMA warp may compute the next stage into it
+            tc_fence_before();
+            mbar_arrive(s_free);
+            const int nvalid = N - j * BN;
+            if (nvalid < BN) {
 #pragma unroll
-                for (int q = 0; q < CW32; ++q)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (32 * q + i >= nvalid) sr[q][i] = __float_as_uint(-INFINITY);
+                for (int k = 0; k < BN; ++k)
+                    if (k >= nvalid) sr[k] = __float_as_uint(-INFINITY);
             }
-            // partial row max of this warp's columns: a tree of three-input maxima
-            float a[CW / 8];
+            // row max of the stage: a tree of three-input maxima
+            float a[BN / 8];
 #pragma unroll
-            for (int k = 0; k < CW / 8; ++k) {
-                const uint32_t* v = &sr[k >> 2][(k & 3) * 8];
-                a[k] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+            for (int g = 0; g < BN / 8; ++g) {
+                const uint32_t* v = &sr[8 * g];
+                a[g] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
                              fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
                              fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
             }
-            float pmax = a[0];
-#pragma unroll
-            for (int k = 1; k < CW / 8; ++k) pmax = fmaxf(pmax, a[k]);
-            // exchange with the other column groups of the same rows (after this
-            // every S read of the tile is done, so P may overwrite S)
-            sm.red_max[b][grp][row] = pmax;
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.bar_group[quad][b]));
-            if (!warp_wait(smem_u32(&sm.bar_group[quad][b]), (j >> 1) & 1, abort_flag, p.status, limit)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            float tmax = sm.red_max[b][0][row];
-#pragma unroll
-            for (int g = 1; g < COL_GROUPS; ++g) tmax = fmaxf(tmax, sm.red_max[b][g][row]);
-            const float mx = tmax * c;
-            float alpha = 1.0f;
-            bool rescale = false;
-            if (mx > m_run + 8.0f) {
-                alpha = ex2_approx(m_run - mx);
-                m_run = mx;
-                rescale = true;
+            static_assert(BN / 8 == 14, "max tree below covers 14 groups");
+            const float mx = fmax3(fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], a[8])),
+                                   fmax3(a[9], a[10], a[11]), fmaxf(a[12], a[13])) * c;
+            // lazy running max: move it only when the stage exceeds it by more than 8
+            const float m_new = (mx > m_run + 8.0f) ? mx : m_run;
+            const bool moved = m_new != m_run;
+            const float alpha = moved ? ex2_approx(m_run - m_new) : 1.0f;  // 0 on the first stage
+            if (moved) {
                 const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) lacc[k] = __fmul2_rn(lacc[k], a2);
             }
+            m_run = m_new;
             const float2 negm = make_float2(-m_run, -m_run);
-            uint32_t pk[CW / 2];
+            uint32_t pk[BN / 2];
 #pragma unroll
-            for (int k = 0; k < CW / 2; ++k) {
-                const float2 s2 = make_float2(__uint_as_float(sr[k >> 4][(2 * k) & 31]),
-                                              __uint_as_float(sr[k >> 4][(2 * k + 1) & 31]));
+            for (int k = 0; k < BN / 2; ++k) {
+                const float2 s2 = make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
                 const float2 x = __ffma2_rn(s2, c2, negm);
                 float2 pv;
                 if ((k & 7) < POLY_PAIRS_PER_8) {
@@ -438,82 +536,67 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 lacc[k & 3] = __fadd2_rn(lacc[k & 3], pv);
                 pk[k] = pack_bf16x2(pv.x, pv.y);
             }
-            // P (bf16 pairs) over this warp's CW/2 columns of the S buffer
-            if constexpr (CW == 64) {
-                tmem_st32(s_addr + 32u * grp, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-            } else {
-                tmem_st16(s_addr + 16u * grp, pk);
-            }
-            tmem_wait_st();
-            // tcgen05.ld/st are warp-collective: the whole warp takes this branch
-            // when any of its rows needs it (alpha is 1 elsewhere).  Only then
-            // does it wait for tile j-1's P.V: S(j) being ready means every
-            // earlier P.V has completed, so that is the only one in flight and
-            // the parity wait is unambiguous.
-            if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
-                if (!warp_wait(smem_u32(&sm.bar_o_done), (j - 1) & 1, abort_flag, p.status, limit)) {
+            if (j > 0) {
+                // the previous P_i V has completed: its P buffer is free and O_i
+                // holds every earlier stage
+                if (!warp_wait(pv_done, (j - 1) & 1, abort_flag, p.status, limit)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t o_addr = tmem + lane_base + TM_O + (uint32_t)(CW * grp);
-                const float2 a2 = make_float2(alpha, alpha);
+                // rescale O_i when any row of the warp moved its max (whole warp:
+                // tcgen05.ld/st are warp-collective; alpha is 1 for other rows)
+                if (__any_sync(0xffffffffu, moved)) {
+                    tc_fence_after();
+                    const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-                for (int q = 0; q < CW32; ++q) {
-                    uint32_t r[32];
-                    tmem_ld32(o_addr + 32u * q, r);
-                    tmem_wait_ld();
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t r[32];
+                        tmem_ld32(o_addr + 32u * q, r);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float2 o2 =
-                            __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), a2);
-                        r[i] = __float_as_uint(o2.x);
-                        r[i + 1] = __float_as_uint(o2.y);
-                    }
-                    tmem_st32(o_addr + 32u * q, r);
-                }
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.bar_p_ready[b]));
-        }
-        if (ok && T > 0) {
-            // total row sum over the column groups (the group barrier's next phase)
-            const float l_part = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) + (lacc[2].x + lacc[2].y) +
-                                 (lacc[3].x + lacc[3].y);
-            sm.red_sum[grp][row] = l_part;
-            mbar_arrive(smem_u32(&sm.bar_group[quad][T & 1]));
-            ok = warp_wait(smem_u32(&sm.bar_group[quad][T & 1]), (T >> 1) & 1, abort_flag, p.status, limit);
-            float l = sm.red_sum[0][row];
-#pragma unroll
-            for (int g = 1; g < COL_GROUPS; ++g) l += sm.red_sum[g][row];
-            if (ok && warp_wait(smem_u32(&sm.bar_o_final), 0, abort_flag, p.status, limit)) {
-                tc_fence_after();
-                const float inv_l = 1.0f / l;
-                const uint32_t o_addr = tmem + lane_base + TM_O + (uint32_t)(CW * grp);
-                const int n = q0 + row;
-                const size_t orow = (size_t)bh * N + n;
-#pragma unroll
-                for (int q = 0; q < CW32; ++q) {
-                    uint32_t r[32];
-                    tmem_ld32(o_addr + 32u * q, r);
-                    tmem_wait_ld();
-                    if (n < N) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + CW * grp + 32 * q);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i = 8 * v + 2 * e;
-                                w[e] = pack_bf16x2(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l);
-                            }
-                            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                        for (int k = 0; k < 32; k += 2) {
+                            const float2 o2 =
+                                __fmul2_rn(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), a2);
+                            r[k] = __float_as_uint(o2.x);
+                            r[k + 1] = __float_as_uint(o2.y);
                         }
+                        tmem_st32(o_addr + 32u * q, r);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                }
+            }
+            store_p_row<BN / 16>(p_tile, row, pk);
+            fence_proxy_async_smem();  // P is read by the tensor cores (async proxy)
+            mbar_arrive(p_full);
+        }
+        if (ok && T > 0 && warp_wait(pv_done, (T - 1) & 1, abort_flag, p.status, limit)) {
+            tc_fence_after();
+            const float l = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) + (lacc[2].x + lacc[2].y) +
+                            (lacc[3].x + lacc[3].y);
+            const float inv_l = 1.0f / l;
+            const int n = q0 + BM * qt + row;
+            const size_t orow = (size_t)bh * N + n;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+                tmem_ld32(o_addr + 32u * q, r);
+                tmem_wait_ld();
+                if (n < N) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + 32 * q);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int k = 8 * v + 2 * e;
+                            w[e] = pack_bf16x2(__uint_as_float(r[k]) * inv_l, __uint_as_float(r[k + 1]) * inv_l);
+                        }
+                        dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
-                if (p.lse && n < N && grp == 0) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
             }
+            if (p.lse && n < N) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
         }
     }
 
@@ -526,11 +609,18 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 }
 
 // ------------------------------------------------------------- probes ----
+// One 128x128 tile through the forward kernel's MMA helpers, descriptors,
+// P layout and scale-factor staging (with N = 128 keys).  TMEM: S [128,256),
+// O [256,384), scale factors of Q [384,392) and of K [392,400).
+
+constexpr uint32_t PR_S = 128, PR_O = 256, PR_SFQ = 384, PR_SFK = 392;
+constexpr uint32_t PR_V_PANEL_BYTES = 128 * 64 * 2;
 
 struct ProbeSmem {
-    uint8_t v[V_TILE_BYTES];
-    uint8_t kc[CODE_TILE_BYTES];
-    uint8_t qc[CODE_TILE_BYTES];
+    uint8_t v[2 * PR_V_PANEL_BYTES];
+    uint8_t pb[8 * P_PANEL_BYTES];
+    uint8_t kc[Q_TILE_BYTES];
+    uint8_t qc[Q_TILE_BYTES];
     uint8_t ks_atom[2][512];
     uint8_t qs_atom[2][512];
     uint64_t bar_full;
@@ -572,30 +662,26 @@ __global__ void __launch_bounds__(160, 1)
     }
     if (threadIdx.x == 128) {
         if (mode == 0) {
-            mbar_arrive_expect_tx(full, 2 * CODE_TILE_BYTES);
+            mbar_arrive_expect_tx(full, 2 * Q_TILE_BYTES);
             tma_load_3d(smem_u32(sm.qc), &tm_qc, 0, 0, 0, full);
             tma_load_3d(smem_u32(sm.kc), &tm_kc, 0, 0, 0, full);
         } else {
-            mbar_arrive_expect_tx(full, V_TILE_BYTES);
+            mbar_arrive_expect_tx(full, 2 * PR_V_PANEL_BYTES);
             tma_load_3d(smem_u32(sm.v), &tm_v, 0, 0, 0, full);
-            tma_load_3d(smem_u32(sm.v) + V_PANEL_BYTES, &tm_v, 64, 0, 0, full);
+            tma_load_3d(smem_u32(sm.v) + PR_V_PANEL_BYTES, &tm_v, 64, 0, 0, full);
         }
     }
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
     if (mode == 1 && warp < 4) {
-        // write P into TMEM exactly as the softmax warps do
+        // write P into shared memory exactly as the softmax warps do (bf16 pairs)
         const int row = 32 * warp + lane;
         const uint32_t* src = reinterpret_cast<const uint32_t*>(pbf + (size_t)row * 128);
-        uint32_t pk[2][32];
+        uint32_t pk[64];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            pk[0][i] = src[i];
-            pk[1][i] = src[32 + i];
-        }
-        tmem_st32(tmem + lane_base + TM_S0, pk[0]);
-        tmem_st32(tmem + lane_base + TM_S0 + 32u, pk[1]);
-        tmem_wait_st();
+        for (int i = 0; i < 64; ++i) pk[i] = src[i];
+        store_p_row<8>(sm.pb, row, pk);
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -605,13 +691,13 @@ __global__ void __launch_bounds__(160, 1)
             if (lane == 0) {
                 tc_fence_after();
                 if (mode == 0) {
-                    tmem_cp_32x128b_x4(tmem + TM_SFQ, atom_desc(sm.qs_atom[0]));
-                    tmem_cp_32x128b_x4(tmem + TM_SFQ + 4, atom_desc(sm.qs_atom[1]));
-                    tmem_cp_32x128b_x4(tmem + TM_SFK, atom_desc(sm.ks_atom[0]));
-                    tmem_cp_32x128b_x4(tmem + TM_SFK + 4, atom_desc(sm.ks_atom[1]));
-                    issue_qk(tmem, TM_S0 + 128u, sm.qc, sm.kc, TM_SFK);
+                    tmem_cp_32x128b_x4(tmem + PR_SFQ, atom_desc(sm.qs_atom[0]));
+                    tmem_cp_32x128b_x4(tmem + PR_SFQ + 4, atom_desc(sm.qs_atom[1]));
+                    tmem_cp_32x128b_x4(tmem + PR_SFK, atom_desc(sm.ks_atom[0]));
+                    tmem_cp_32x128b_x4(tmem + PR_SFK + 4, atom_desc(sm.ks_atom[1]));
+                    issue_qk(tmem, PR_S, sm.qc, sm.kc, PR_SFQ, PR_SFK, idesc_qk(128));
                 } else {
-                    issue_pv(tmem, TM_S0, sm.v, false);
+                    issue_pv<128>(tmem, PR_O, sm.pb, sm.v, PR_V_PANEL_BYTES, false);
                 }
             }
         }
@@ -620,7 +706,7 @@ __global__ void __launch_bounds__(160, 1)
     }
     if (warp < 4) {
         const int row = 32 * warp + lane;
-        const uint32_t col = (mode == 0) ? TM_S0 + 128u : TM_O;
+        const uint32_t col = (mode == 0) ? PR_S : PR_O;
         if (warp_wait(smem_u32(&sm.bar_done), 0, abort_flag, status, kWaitLimitNs)) {
             tc_fence_after();
 #pragma unroll
@@ -662,21 +748,21 @@ struct Maps {
     CUtensorMap qc, kc, v;
 };
 
-// Codes [BH][N][64 bytes]: 64B-swizzled boxes of 128 rows; x is always 0.
-bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N) {
+// Codes [BH][N][64 bytes]: 64B-swizzled boxes of box_rows rows; x is always 0.
+bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N, uint32_t box_rows) {
     const uint64_t dims[3] = {64, (uint64_t)N, (uint64_t)BH};
     const uint64_t strides[2] = {64, (uint64_t)N * 64};
-    const uint32_t box[3] = {64, 128, 1};
+    const uint32_t box[3] = {64, box_rows, 1};
     return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims,
                              strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// V [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x 128 keys; x is 0 or 64
-// (0 or 128 bytes), so every box starts on a 16-byte boundary.
-bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N) {
+// V [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x box_rows keys; x is
+// 0 or 64 (0 or 128 bytes), so every box starts on a 16-byte boundary.
+bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N, uint32_t box_rows) {
     const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH};
     const uint64_t strides[2] = {256, (uint64_t)N * 256};
-    const uint32_t box[3] = {64, 128, 1};
+    const uint32_t box[3] = {64, box_rows, 1};
     return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(base),
                              dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
@@ -689,8 +775,8 @@ size_t probe_smem_bytes() { return sizeof(ProbeSmem) + 1024; }
 int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     Maps m;
-    if (!make_code_map(&m.qc, a.q_codes, a.BH, a.N) || !make_code_map(&m.kc, a.k_codes, a.BH, a.N) ||
-        !make_v_map(&m.v, a.v, a.BH, a.N))
+    if (!make_code_map(&m.qc, a.q_codes, a.BH, a.N, BM) || !make_code_map(&m.kc, a.k_codes, a.BH, a.N, BN) ||
+        !make_v_map(&m.v, a.v, a.BH, a.N, BN))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(FwdSmem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = fwd_smem_bytes();
@@ -710,7 +796,7 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     p.lse = a.lse;
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;
-    dim3 grid((a.N + BM - 1) / BM, a.BH);
+    dim3 grid((a.N + QT * BM - 1) / (QT * BM), a.BH);
     fwd_kernel<<<grid, FWD_THREADS, smem, stream>>>(m.qc, m.kc, m.v, p);
     return cudaGetLastError() == cudaSuccess ? FP4ATTN_OK : FP4ATTN_ERR_CUDA;
 }
@@ -720,10 +806,11 @@ static int launch_probe(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc,
                         cudaStream_t stream) {
     Maps m;
     if (mode == 0) {
-        if (!make_code_map(&m.qc, qc, 1, 128) || !make_code_map(&m.kc, kc, 1, 128)) return FP4ATTN_ERR_CUDA;
+        if (!make_code_map(&m.qc, qc, 1, 128, 128) || !make_code_map(&m.kc, kc, 1, 128, 128))
+            return FP4ATTN_ERR_CUDA;
         m.v = m.qc;  // unused in this mode
     } else {
-        if (!make_v_map(&m.v, v, 1, 128)) return FP4ATTN_ERR_CUDA;
+        if (!make_v_map(&m.v, v, 1, 128, 128)) return FP4ATTN_ERR_CUDA;
         m.qc = m.kc = m.v;  // unused in this mode
     }
     const size_t smem = probe_smem_bytes();
