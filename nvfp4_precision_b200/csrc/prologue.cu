@@ -12,19 +12,25 @@
 //                  round_half_even(k * 2^24)); order-independent, so atomics
 //                  give the same bits as any serial order; then the head's
 //                  ready counter is bumped;
-//   Q / K tile     one thread per 128-channel row: bf16 -> fp32, (K) minus the
-//                  head mean once the head's counter is complete, the 7
-//                  butterfly stages of the Walsh-Hadamard transform in
-//                  registers, x fp32(1/sqrt(128)), per-16 amax, UE4M3 scale
-//                  amax/6/g, E2M1 codes of y * (1/(g*scale)).
+//   Q / K tile     two threads per 128-channel row: bf16 -> fp32, (K) minus
+//                  the head mean once the head's counter is complete, the 7
+//                  butterfly stages of the Walsh-Hadamard transform,
+//                  x fp32(1/sqrt(128)), per-16 amax, UE4M3 scale amax/6/g,
+//                  E2M1 codes of y * (1/(g*scale)).
 // The Q tiles of a head sit between its key-sum and K tiles, so the second
 // read of K mostly hits L2 (key-sum loads are marked evict-last, the others
-// evict-first).  Tiles arrive by TMA (128B swizzle) into a double buffer while
-// the previous tile is computed.  A row's 128 values live in registers as 64
-// pairs (x_i, x_{i+64}): the butterfly stages of stride 1..32 run on packed
-// fp32x2 instructions, the stride-64 stage inside each pair.  Every fp32 step
-// is an explicit round-to-nearest operation, so the codes are bit-identical to
-// the plain CPU definition of the same steps.
+// evict-first).  Tiles arrive by TMA (128B swizzle) in a ring of NBUF buffers
+// per CTA.  Each tile is first copied from its buffer into registers; after
+// one barrier the buffer is refilled with the tile NBUF tickets ahead, so every
+// buffer is in flight while a tile is computed.
+//
+// A row's 128 values live in the registers of two neighbouring lanes as pairs
+// (x_i, x_{i+64}), lane h holding i in [32h, 32h+32): the butterfly stages of
+// stride 1..16 run on packed fp32x2 instructions inside a lane, stride 32
+// between the two lanes (one shuffle per value), stride 64 inside each pair.
+// Every fp32 step is an explicit round-to-nearest operation applied in the
+// same stage order as the plain CPU definition, so the codes are bit-identical
+// to it.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -36,20 +42,22 @@ namespace {
 
 constexpr float kTwo24 = 16777216.0f;
 constexpr float kKeyLimit = 1048576.0f;  // |k| < 2^20 keeps the int64 sum exact for N <= 2^18
-constexpr int PRO_THREADS = 128;         // one thread per row of a tile
+constexpr int PRO_THREADS = 256;         // two threads per row of a 128-row tile
 constexpr uint32_t HALF_BYTES = 128 * 128;        // 128 rows x 64 channels bf16
 constexpr uint32_t TILE_BYTES = 2 * HALF_BYTES;   // 32 KB
 constexpr uint64_t kSpinLimitNs = 2000000000ull;
 
 enum TileKind { KIND_KSUM = 0, KIND_Q = 1, KIND_K = 2 };
 
+constexpr int NBUF = 3;  // tile ring depth: NBUF-1 tiles in flight while one is computed
+
 struct __align__(1024) ProSmem {
-    uint8_t tile[2][TILE_BYTES];   // double buffer; channels 0-63 then 64-127, 128B swizzle
-    long long part[2][128];        // key-sum partials of even / odd rows
-    float2 neg_mean2[64];          // (-m_i, -m_{i+64})
-    float inv_scale[128];          // fp32 1 / value of each UE4M3 code (0 for code 0)
-    uint64_t bar[2];
-    int next_ticket[2];
+    uint8_t tile[NBUF][TILE_BYTES];  // channels 0-63 then 64-127, 128B swizzle
+    long long kpart[PRO_THREADS / 32][128];  // key-sum partials of the warps
+    float2 neg_mean2[64];            // (-m_i, -m_{i+64})
+    float inv_scale[128];            // fp32 1 / value of each UE4M3 code (0 for code 0)
+    uint64_t bar[NBUF];
+    int next_ticket[NBUF];
     int mean_head;
     int abort_flag;
 };
@@ -126,7 +134,7 @@ __device__ __forceinline__ void block_scale(float a, float g, bool g_is_one, con
     }
 }
 
-__global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                const __grid_constant__ CUtensorMap tm_k,
                                                                const ProArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -140,26 +148,21 @@ __global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_cons
     const int total = a.BH * per_head;
 
     if (tid == 0) {
-        mbar_init(smem_u32(&sm.bar[0]), 1);
-        mbar_init(smem_u32(&sm.bar[1]), 1);
+        for (int b = 0; b < NBUF; ++b) mbar_init(smem_u32(&sm.bar[b]), 1);
         sm.mean_head = -1;
         sm.abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
     }
-    {
-        const float sd = ue4m3_value(tid);  // tid < 128 covers every code; 127 (NaN) is never produced
+    if (tid < 128) {
+        const float sd = ue4m3_value(tid);  // codes 0..127 cover every scale; 127 (NaN) is never produced
         sm.inv_scale[tid] = (sd != 0.0f) ? __frcp_rn(sd) : 0.0f;
     }
-    float g[2] = {1.0f, 1.0f};
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-        if (a.g[w]) {
-            g[w] = *a.g[w];
-            if (!(g[w] > 0.0f && g[w] < INFINITY) && tid == 0) set_status(a.status, FP4ATTN_ERR_RANGE);
-        }
-    }
+    float gq = 1.0f, gk = 1.0f;
+    if (a.g[0]) gq = *a.g[0];
+    if (a.g[1]) gk = *a.g[1];
+    if (tid == 0 && !(gq > 0.0f && gq < INFINITY && gk > 0.0f && gk < INFINITY)) set_status(a.status, FP4ATTN_ERR_RANGE);
     __syncthreads();
 
     const uint64_t pol_keep = l2_policy_evict_last();
@@ -181,64 +184,85 @@ __global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_cons
         tma_load_3d_hint(smem_u32(sm.tile[buf]) + HALF_BYTES, map, 64, tile * 128, bh, bar, pol);
     };
 
-    bool in_flight[2] = {false, false};  // tracked by thread 0, which issues the copies
+    uint32_t in_flight = 0u;  // bit b: a copy into buffer b is outstanding (thread 0, which issues them)
     if (tid == 0) {
-        const int t0 = (int)atomicAdd(a.ticket, 1u);
-        sm.next_ticket[0] = t0;
-        if (t0 < total) {
-            issue(t0, 0);
-            in_flight[0] = true;
+        for (int b = 0; b < NBUF; ++b) {
+            const int tk = (int)atomicAdd(a.ticket, 1u);
+            sm.next_ticket[b] = tk;
+            if (tk < total) {
+                issue(tk, b);
+                in_flight |= 1u << b;
+            }
         }
     }
     __syncthreads();
     int t = sm.next_ticket[0];
     int buf = 0;
-    uint32_t phase[2] = {0u, 0u};
+    uint32_t phase = 0u;  // bit b: parity of the next phase of buffer b
 
-    while (t < total) {
-        // prefetch the next tile into the other buffer
+    // Each tile is first copied from its buffer into registers; after one barrier
+    // the buffer is refilled with the tile NBUF iterations ahead, so all NBUF
+    // buffers are in flight while the tile is computed.
+    auto release = [&](int b) {  // after the barrier that ends the reads of buffer b
         if (tid == 0) {
             const int tn = (int)atomicAdd(a.ticket, 1u);
-            sm.next_ticket[buf ^ 1] = tn;
+            sm.next_ticket[b] = tn;
             if (tn < total) {
-                issue(tn, buf ^ 1);
-                in_flight[buf ^ 1] = true;
+                issue(tn, b);
+                in_flight |= 1u << b;
             }
         }
+    };
+    while (t < total) {
         int kind, bh, tile;
         decode(t, kind, bh, tile);
-        const bool landed = mbar_wait(smem_u32(&sm.bar[buf]), phase[buf], &sm.abort_flag, a.status, kSpinLimitNs);
+        const bool landed = mbar_wait(smem_u32(&sm.bar[buf]), (phase >> buf) & 1u, &sm.abort_flag, a.status, kSpinLimitNs);
         if (__syncthreads_or(!landed)) break;
-        phase[buf] ^= 1u;
-        in_flight[buf] = false;
+        phase ^= 1u << buf;
+        in_flight &= ~(1u << buf);
         const uint8_t* tb = sm.tile[buf];
 
         if (kind == KIND_KSUM) {
             // ------------------------------------------------ key sums ----
-            const int cp = tid & 63;       // channel pair (2cp, 2cp+1)
-            const int rpar = tid >> 6;     // rows of this parity
-            const uint8_t* hb = tb + (cp >> 5) * HALF_BYTES;
-            const int j = (cp & 31) >> 2;
-            const uint32_t in_chunk = (uint32_t)(cp & 3) * 4u;
-            long long acc0 = 0, acc1 = 0;
+            // warp w: rows 16w..16w+15; lane l: channels 4l..4l+3 (one 8-byte load
+            // per row), four independent int64 accumulators
+            const int warp = tid >> 5, lane = tid & 31;
+            const uint8_t* hb = tb + (lane >> 4) * HALF_BYTES;
+            const int j = (lane & 15) >> 1;
+            const uint32_t in_chunk = (uint32_t)(lane & 1) * 8u;
+            uint2 kw[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) kw[rr] = *reinterpret_cast<const uint2*>(hb + swz(16 * warp + rr, j) + in_chunk);
+            __syncthreads();
+            release(buf);
+            long long acc[4] = {0, 0, 0, 0};
             bool bad = false;
-#pragma unroll 8
-            for (int r = rpar; r < 128; r += 2) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(hb + swz(r, j) + in_chunk);
-                const float v0 = bf16lo(w), v1 = bf16hi(w);
-                if (fabsf(v0) < kKeyLimit) acc0 += __float2ll_rn(__fmul_rn(v0, kTwo24)); else bad = true;
-                if (fabsf(v1) < kKeyLimit) acc1 += __float2ll_rn(__fmul_rn(v1, kTwo24)); else bad = true;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const float v[4] = {bf16lo(kw[rr].x), bf16hi(kw[rr].x), bf16lo(kw[rr].y), bf16hi(kw[rr].y)};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (fabsf(v[c]) < kKeyLimit) acc[c] += __float2ll_rn(__fmul_rn(v[c], kTwo24)); else bad = true;
+                }
             }
             if (bad) set_status(a.status, FP4ATTN_ERR_RANGE);
-            sm.part[rpar][2 * cp] = acc0;
-            sm.part[rpar][2 * cp + 1] = acc1;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sm.kpart[warp][4 * lane + c] = acc[c];
             __syncthreads();
-            const long long tot = sm.part[0][tid] + sm.part[1][tid];
-            atomicAdd(reinterpret_cast<unsigned long long*>(a.ksum + (size_t)bh * D + tid),
-                      static_cast<unsigned long long>(tot));
-            __threadfence();
+            if (tid < 128) {
+                long long tot = 0;
+#pragma unroll
+                for (int w = 0; w < PRO_THREADS / 32; ++w) tot += sm.kpart[w][tid];
+                atomicAdd(reinterpret_cast<unsigned long long*>(a.ksum + (size_t)bh * D + tid),
+                          static_cast<unsigned long long>(tot));
+            }
+            // the CTA barrier makes every thread's sum visible to thread 0, whose
+            // device-scope fence then orders them all before the ready count
             __syncthreads();
-            if (tid == 0) atomicAdd(a.head_ready + bh, 1u);
+            if (tid == 0) {
+                __threadfence();
+                atomicAdd(a.head_ready + bh, 1u);
+            }
         } else {
             const int which = kind - 1;  // 0 = Q, 1 = K
             if (which == 1 && sm.mean_head != bh) {
@@ -258,27 +282,39 @@ __global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_cons
                     __threadfence();
                 }
                 if (__syncthreads_or(!ready)) break;
-                float m = 0.0f;
-                if (smooth) {
-                    const long long S = __ldcg(a.ksum + (size_t)bh * D + tid);
-                    m = __double2float_rn(__ddiv_rn(__ll2double_rn(S), (double)N * 16777216.0));
+                if (tid < 128) {
+                    float m = 0.0f;
+                    if (smooth) {
+                        const long long S = __ldcg(a.ksum + (size_t)bh * D + tid);
+                        m = __double2float_rn(__ddiv_rn(__ll2double_rn(S), (double)N * 16777216.0));
+                    }
+                    if (tid < 64) sm.neg_mean2[tid].x = -m; else sm.neg_mean2[tid - 64].y = -m;
+                    if (a.k_mean && tile == 0) a.k_mean[(size_t)bh * D + tid] = m;
                 }
-                if (tid < 64) sm.neg_mean2[tid].x = -m; else sm.neg_mean2[tid - 64].y = -m;
-                if (a.k_mean && tile == 0) a.k_mean[(size_t)bh * D + tid] = m;
                 __syncthreads();
                 if (tid == 0) sm.mean_head = bh;
             }
             // ---------------------------------------------- one row ----
-            const int r = tid;
-            float2 P[64];  // P[i] = (x_i, x_{i+64})
+            // lanes 2r', 2r'+1 of a warp share row r; lane half h holds the pairs
+            // P[k] = (x_i, x_{i+64}), i = 32h + k
+            const int r = tid >> 1;
+            const int h = tid & 1;
+            float2 P[32];
             const bool sub_mean = (which == 1) && smooth;
             bool finite = true;
-            // chunk j holds pairs 8j..8j+7: load, unpack, smooth, and apply the
+            uint4 rlo[4], rhi[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                rlo[j] = *reinterpret_cast<const uint4*>(tb + swz(r, 4 * h + j));
+                rhi[j] = *reinterpret_cast<const uint4*>(tb + HALF_BYTES + swz(r, 4 * h + j));
+            }
+            __syncthreads();
+            release(buf);
+            // chunk j (8 pairs, k = 8j..8j+7): unpack, smooth, and apply the
             // butterfly stages of stride 1, 2, 4, which stay inside the chunk
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint4 lo = *reinterpret_cast<const uint4*>(tb + swz(r, j));
-                const uint4 hi = *reinterpret_cast<const uint4*>(tb + HALF_BYTES + swz(r, j));
+            for (int j = 0; j < 4; ++j) {
+                const uint4 lo = rlo[j], hi = rhi[j];
                 const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
                 const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
                 float2* C = P + 8 * j;
@@ -288,7 +324,7 @@ __global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_cons
                     C[2 * e + 1] = f2(bf16hi(wl[e]), bf16hi(wh[e]));
                 }
                 if (sub_mean) {
-                    const float4* nm = reinterpret_cast<const float4*>(sm.neg_mean2 + 8 * j);
+                    const float4* nm = reinterpret_cast<const float4*>(sm.neg_mean2 + 32 * h + 8 * j);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float4 m4 = nm[e];
@@ -301,84 +337,96 @@ __global__ void __launch_bounds__(PRO_THREADS) prologue_kernel(const __grid_cons
                     for (int i = 0; i < 8; ++i) finite &= (fabsf(C[i].x) < INFINITY) && (fabsf(C[i].y) < INFINITY);
                 } else {
 #pragma unroll
-                    for (int h = 1; h < 8; h <<= 1) {
+                    for (int st = 1; st < 8; st <<= 1) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            if ((i & h) == 0) {
-                                const float2 x = C[i], y = C[i + h];
+                            if ((i & st) == 0) {
+                                const float2 x = C[i], y = C[i + st];
                                 C[i] = __fadd2_rn(x, y);
-                                C[i + h] = sub2(x, y);
+                                C[i + st] = sub2(x, y);
                             }
                         }
                     }
                 }
             }
             if (hadamard) {
-                // strides 8, 16, 32 across chunks, then 64 inside each pair
+                // strides 8 and 16 across chunks
 #pragma unroll
-                for (int h = 8; h < 64; h <<= 1) {
+                for (int st = 8; st < 32; st <<= 1) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        if ((i & h) == 0) {
-                            const float2 x = P[i], y = P[i + h];
+                    for (int i = 0; i < 32; ++i) {
+                        if ((i & st) == 0) {
+                            const float2 x = P[i], y = P[i + st];
                             P[i] = __fadd2_rn(x, y);
-                            P[i + h] = sub2(x, y);
+                            P[i + st] = sub2(x, y);
                         }
                     }
                 }
+                // stride 32 between the two lanes of the row: lane 0 keeps
+                // x_i + x_{i+32}, lane 1 keeps x_i - x_{i+32}
+                const float sg = h ? -1.0f : 1.0f;  // fl(other + sg * own): the sum or the difference, one rounding
 #pragma unroll
-                for (int i = 0; i < 64; ++i) P[i] = f2(__fadd_rn(P[i].x, P[i].y), __fsub_rn(P[i].x, P[i].y));
-                // y_0 is the sum of all 128 inputs: it is finite iff they all are
-                // (barring overflow of the sum itself)
-                finite = fabsf(P[0].x) < INFINITY;
+                for (int k = 0; k < 32; ++k) {
+                    const float ox = __shfl_xor_sync(0xffffffffu, P[k].x, 1);
+                    const float oy = __shfl_xor_sync(0xffffffffu, P[k].y, 1);
+                    P[k] = __ffma2_rn(P[k], f2(sg, sg), f2(ox, oy));
+                }
+                // stride 64 inside each pair
+#pragma unroll
+                for (int k = 0; k < 32; ++k) P[k] = f2(__fadd_rn(P[k].x, P[k].y), __fsub_rn(P[k].x, P[k].y));
+                // y_0 (lane 0, P[0].x) is the sum of all 128 inputs: it is finite iff
+                // they all are (barring overflow of the sum itself)
+                finite = (h != 0) || (fabsf(P[0].x) < INFINITY);
                 const float c = __uint_as_float(0x3DB504F3u);  // fp32(1/sqrt(128))
 #pragma unroll
-                for (int i = 0; i < 64; ++i) P[i] = __fmul2_rn(P[i], f2(c, c));
+                for (int k = 0; k < 32; ++k) P[k] = __fmul2_rn(P[k], f2(c, c));
             }
 
-            // NVFP4 pack.  Blocks 0-3 are the .x lanes of P[0..63], blocks 4-7
-            // the .y lanes; block b's codes are words 2b, 2b+1 of the row.
-            const float gw = g[which];
+            // NVFP4 pack.  This lane holds blocks 2h, 2h+1 (the .x lanes of
+            // P[0..15], P[16..31]) and 4+2h, 5+2h (the .y lanes); block b's codes
+            // are bytes 8b..8b+7 of the row.
+            const float gw = which ? gk : gq;
             const bool g_is_one = (gw == 1.0f);
             const bool valid = (tile * 128 + r) < N;
             if (!finite && valid) set_status(a.status, FP4ATTN_ERR_RANGE);
             const size_t row = (size_t)bh * N + (size_t)tile * 128 + r;
-            uint4* dst = reinterpret_cast<uint4*>(a.codes[which] + row * 64);
-            uint32_t lo[4], hi[4];  // code words of blocks (bb-1, bb) and (bb+3, bb+4)
-            uint32_t sw_lo = 0, sw_hi = 0;
+            uint32_t s_b[4];  // scale bytes of blocks 2h, 2h+1, 4+2h, 5+2h
+            uint32_t w_lo[4], w_hi[4];
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                uint32_t s_lo, s_hi;
+            for (int bb = 0; bb < 2; ++bb) {
                 float inv_lo, inv_hi;
-                block_scale(amax16(P + 16 * bb, false), gw, g_is_one, sm.inv_scale, s_lo, inv_lo);
-                block_scale(amax16(P + 16 * bb, true), gw, g_is_one, sm.inv_scale, s_hi, inv_hi);
-                sw_lo |= s_lo << (8 * bb);
-                sw_hi |= s_hi << (8 * bb);
+                block_scale(amax16(P + 16 * bb, false), gw, g_is_one, sm.inv_scale, s_b[bb], inv_lo);
+                block_scale(amax16(P + 16 * bb, true), gw, g_is_one, sm.inv_scale, s_b[2 + bb], inv_hi);
                 const float2 inv2 = f2(inv_lo, inv_hi);
 #pragma unroll
                 for (int h8 = 0; h8 < 2; ++h8) {
                     float2 R[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) R[k] = __fmul2_rn(P[16 * bb + 8 * h8 + k], inv2);
-                    lo[2 * (bb & 1) + h8] = cvt_e2m1x8(R[0].x, R[1].x, R[2].x, R[3].x, R[4].x, R[5].x, R[6].x, R[7].x);
-                    hi[2 * (bb & 1) + h8] = cvt_e2m1x8(R[0].y, R[1].y, R[2].y, R[3].y, R[4].y, R[5].y, R[6].y, R[7].y);
-                }
-                if ((bb & 1) && valid) {
-                    dst[bb >> 1] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                    dst[2 + (bb >> 1)] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    w_lo[2 * bb + h8] = cvt_e2m1x8(R[0].x, R[1].x, R[2].x, R[3].x, R[4].x, R[5].x, R[6].x, R[7].x);
+                    w_hi[2 * bb + h8] = cvt_e2m1x8(R[0].y, R[1].y, R[2].y, R[3].y, R[4].y, R[5].y, R[6].y, R[7].y);
                 }
             }
-            if (valid) *reinterpret_cast<uint2*>(a.scales[which] + row * 8) = make_uint2(sw_lo, sw_hi);
+            // scale bytes: lane 0 writes blocks 0-3, lane 1 blocks 4-7
+            const uint32_t mine_lo = s_b[0] | (s_b[1] << 8), mine_hi = s_b[2] | (s_b[3] << 8);
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, h ? mine_lo : mine_hi, 1);
+            const uint32_t sword = h ? (other | (mine_hi << 16)) : (mine_lo | (other << 16));
+            if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>((which ? a.codes[1] : a.codes[0]) + row * 64);
+                dst[h] = make_uint4(w_lo[0], w_lo[1], w_lo[2], w_lo[3]);
+                dst[2 + h] = make_uint4(w_hi[0], w_hi[1], w_hi[2], w_hi[3]);
+                *reinterpret_cast<uint32_t*>((which ? a.scales[1] : a.scales[0]) + row * 8 + 4 * h) = sword;
+            }
         }
-        __syncthreads();  // tile[buf] is free; next_ticket[buf ^ 1] is visible
-        t = sm.next_ticket[buf ^ 1];
-        buf ^= 1;
+        // the next buffer's ticket was written at least one barrier ago
+        buf = (buf + 1) % NBUF;
+        t = sm.next_ticket[buf];
     }
     // wind down after an abort: let this CTA's own copies land before exiting
     if (tid == 0) {
         int dummy = 0;
-        for (int b = 0; b < 2; ++b)
-            if (in_flight[b]) mbar_wait(smem_u32(&sm.bar[b]), phase[b], &dummy, nullptr, 200000000ull);
+        for (int b = 0; b < NBUF; ++b)
+            if (in_flight & (1u << b)) mbar_wait(smem_u32(&sm.bar[b]), (phase >> b) & 1u, &dummy, nullptr, 200000000ull);
     }
 }
 
