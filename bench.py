@@ -40,10 +40,15 @@ METRIC = "FP4-attn TFLOPS @N=109k,d=128 (% composite roofline); quantize GB/s"
 UNIT = "TFLOP/s"
 WORKLOAD = "clip15s"
 PROLOGUE_BYTES_PER_ELEMENT = 5.125  # Q,K bf16 read (2+2) + codes (0.5+0.5) + scales (1/16+1/16)
-# ncu DRAM bytes (read + write) per launch of the attention kernel, keyed by
-# the sha256 of the attention source they were measured on; a changed kernel
-# reports null until it is profiled again.
-ATTN_TRAFFIC_BYTES = {}
+# ncu DRAM bytes (read + write) per launch, keyed by the sha256 prefix of the
+# kernel source they were measured on and the workload; a changed kernel reports
+# null until it is profiled again (profiles/ holds the commands).
+ATTN_TRAFFIC_BYTES = {
+    ("a6a1dd35d211ef39", "clip15s"): 2.40e9 + 1.39e9,
+}
+PROLOGUE_TRAFFIC_BYTES = {
+    ("1eeb4d396cdc574e", "clip15s"): 2.70e9 + 0.725e9,
+}
 
 
 def log(*a):
@@ -312,8 +317,9 @@ def run_ours(args, rank, world, local):
     att_tflops = F / (ms_att_max * 1e-3) / 1e12
     pro_bytes = PROLOGUE_BYTES_PER_ELEMENT * B * H * N * 128
     pro_gbs = pro_bytes / (ms_pro_max * 1e-3) / 1e9
-    att_src = os.path.join(ROOT, "nvfp4_precision_b200", "csrc", "attention.cu")
-    traffic = ATTN_TRAFFIC_BYTES.get(source_hash(att_src))
+    csrc = os.path.join(ROOT, "nvfp4_precision_b200", "csrc")
+    traffic = ATTN_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "attention.cu")), args.workload))
+    pro_traffic = PROLOGUE_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "prologue.cu")), args.workload))
 
     # ---- end to end through the public API: pinned host inputs in, O out ----
     e2e = None
@@ -358,7 +364,7 @@ def run_ours(args, rank, world, local):
                           "frac_composite_sustained": att_tflops / p_comp,
                           "frac_composite_nominal": att_tflops / composite_peak(2250.0)},
             "quantize": {"ms": ms_pro_max, "gbs": pro_gbs, "frac_hbm": pro_gbs / peaks["hbm_gbs"],
-                         "bytes": pro_bytes},
+                         "bytes": pro_bytes, "traffic": pro_traffic},
             "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": p_comp, "unit": "TFLOP/s",
                          "frac": att_tflops / p_comp, "traffic": traffic,
                          "peak_note": (f"composite FP4/BF16 peak from {peaks['source']} sustained bf16 "
