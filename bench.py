@@ -264,7 +264,7 @@ def run_ours(args, rank, world, local):
     o = torch.empty_like(v)
     ws = fa.new_workspace(B, H, N, dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 3  # key sums, quantise, attention
+    launches_per_step = 2  # the fused prologue, the attention
 
     def step(ev=None):
         if ev is not None:
@@ -317,6 +317,26 @@ def run_ours(args, rank, world, local):
     att_tflops = F / (ms_att_max * 1e-3) / 1e12
     pro_bytes = PROLOGUE_BYTES_PER_ELEMENT * B * H * N * 128
     pro_gbs = pro_bytes / (ms_pro_max * 1e-3) / 1e9
+    # ---- the BF16-QK attention on the same inputs (outside the timed step) ----
+    bf16qk = None
+    if not args.no_bf16qk:
+        o2 = torch.empty_like(v)
+        fa.fp4attn_forward_bf16qk(q, k, v, o=o2, workspace=ws, stream=stream)
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for e in bev:
+            e[0].record(stream)
+            fa.fp4attn_forward_bf16qk(q, k, v, o=o2, workspace=ws, stream=stream)
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        st = fa.fp4attn_read_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status after the BF16-QK attention: {fa.status_string(st)}")
+        ms_b = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in bev), world, dev)
+        tf_b = F / (ms_b * 1e-3) / 1e12
+        bf16qk = {"ms": ms_b, "tflops": tf_b, "frac_bf16_sustained": tf_b / peaks["bf16_sustained"],
+                  "fp4_speedup": ms_b / ms_att_max}
+        del o2
+
     csrc = os.path.join(ROOT, "nvfp4_precision_b200", "csrc")
     traffic = ATTN_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "attention.cu")), args.workload))
     pro_traffic = PROLOGUE_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "prologue.cu")), args.workload))
@@ -365,6 +385,7 @@ def run_ours(args, rank, world, local):
                           "frac_composite_nominal": att_tflops / composite_peak(2250.0)},
             "quantize": {"ms": ms_pro_max, "gbs": pro_gbs, "frac_hbm": pro_gbs / peaks["hbm_gbs"],
                          "bytes": pro_bytes, "traffic": pro_traffic},
+            "bf16qk_attention": bf16qk,
             "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": p_comp, "unit": "TFLOP/s",
                          "frac": att_tflops / p_comp, "traffic": traffic,
                          "peak_note": (f"composite FP4/BF16 peak from {peaks['source']} sustained bf16 "
@@ -389,6 +410,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-bf16qk", action="store_true", help="skip timing the BF16-QK attention")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

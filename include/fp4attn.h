@@ -109,6 +109,21 @@ int fp4attn_forward(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
                     void* o_bf16_dev, float* lse_dev,
                     void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
 
+/* The same non-causal attention with Q and K in BF16 instead of NVFP4: the
+ * baseline the FP4 kernel is measured against, and the path for layers kept in
+ * BF16 (FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention": two of
+ * the model's attention blocks stay in BF16).  S = Q K^T runs on the BF16
+ * tensor cores with fp32 accumulation; softmax, P (bf16) and P V are as in
+ * fp4attn_forward.  No smoothing, rotation or quantisation is applied.
+ *   q_bf16_dev, k_bf16_dev, v_bf16_dev : [B,H,N,128] bf16.
+ *   softmax_scale : <= 0 selects 1/sqrt(128).
+ *   o_bf16_dev : [B,H,N,128] out.  lse_dev : [B,H,N] out or NULL.
+ *   workspace_dev : as for fp4attn_forward (status word only; not cleared).
+ * Device errors: FP4ATTN_ERR_TIMEOUT if an internal wait ran out. */
+int fp4attn_forward_bf16qk(const void* q_bf16_dev, const void* k_bf16_dev, const void* v_bf16_dev,
+                           fp4attn_shape s, float softmax_scale, void* o_bf16_dev, float* lse_dev,
+                           void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
+
 /* fp4attn_quantize_qk without a workspace argument.  The pages have no
  * counterpart to this entry point: it exists for callers that cannot allocate
  * device memory for the workspace -- cudaMalloc/cudaFree may synchronise the

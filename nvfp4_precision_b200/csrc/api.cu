@@ -165,6 +165,33 @@ int fp4attn_forward(const uint8_t* q_codes, const uint8_t* q_scales, const uint8
     return st;
 }
 
+int fp4attn_forward_bf16qk(const void* q, const void* k, const void* v, fp4attn_shape s, float softmax_scale,
+                           void* o, float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    int st = check_shape(s);
+    if (st != FP4ATTN_OK) return st;
+    if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
+        return FP4ATTN_ERR_WORKSPACE;
+    if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f) return FP4ATTN_ERR_INVALID_ARG;
+    if (empty(s)) return FP4ATTN_OK;
+    const void* ptrs[] = {q, k, v, o};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
+    if (lse && ((uintptr_t)lse & 3)) return FP4ATTN_ERR_INVALID_ARG;
+    FwdBf16Args a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.BH = (int)heads(s);
+    a.N = s.N;
+    a.softmax_scale = softmax_scale;
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.lse = lse;
+    a.status = static_cast<int*>(workspace);
+    st = launch_forward_bf16qk(a, stream);
+    if (st != FP4ATTN_OK) (void)cudaGetLastError();
+    return st;
+}
+
 int fp4attn_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s,
                     float* out, cudaStream_t stream) {
     int st = check_shape(s);

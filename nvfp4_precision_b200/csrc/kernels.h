@@ -67,8 +67,20 @@ struct FwdArgs {
     int* status;
 };
 
+struct FwdBf16Args {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    int BH, N;
+    float softmax_scale;
+    __nv_bfloat16* o;
+    float* lse;
+    int* status;
+};
+
 // Returns 0 on success, else an fp4attn_status code.
 int launch_forward(const FwdArgs& a, cudaStream_t stream);
+int launch_forward_bf16qk(const FwdBf16Args& a, cudaStream_t stream);
 int launch_probe_qk(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
                     float* s_out, cudaStream_t stream);
 int launch_probe_pv(const __nv_bfloat16* p, const __nv_bfloat16* v, float* o_out,

@@ -28,6 +28,7 @@ NO_HADAMARD = 2
 
 EXPORTS = (
     "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_quantize_qk_noalloc", "fp4attn_forward",
+    "fp4attn_forward_bf16qk",
     "fp4attn_dequant",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
@@ -58,6 +59,8 @@ def _load():
     L.fp4attn_quantize_qk_noalloc.argtypes = [P, P, Shape, P, P, U32, P, P, P, P, P, P, P]
     L.fp4attn_forward.restype = ctypes.c_int
     L.fp4attn_forward.argtypes = [P, P, P, P, P, P, P, Shape, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_forward_bf16qk.restype = ctypes.c_int
+    L.fp4attn_forward_bf16qk.argtypes = [P, P, P, Shape, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
     L.fp4attn_dequant.restype = ctypes.c_int
     L.fp4attn_dequant.argtypes = [P, P, P, Shape, P, P]
     L.fp4attn_read_status.restype = ctypes.c_int
@@ -184,6 +187,27 @@ def fp4attn_forward(q_codes, q_scales, k_codes, k_scales, v: torch.Tensor, q_gsc
                              _ptr(k_gscale), _ptr(v), Shape(B, H, N, D), float(softmax_scale), _ptr(o), _ptr(lse),
                              _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "fp4attn_forward")
+    return o, lse
+
+
+def fp4attn_forward_bf16qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float = 0.0,
+                           o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                           want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Non-causal attention with bf16 Q, K, V [B,H,N,128] (no quantisation): the
+    BF16 counterpart of fp4attn_forward.  Returns (O, lse or None)."""
+    for t in (q, k, v):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == v.shape
+    B, H, N, D = v.shape
+    if o is None:
+        o = torch.empty_like(v)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
+    if workspace is None:
+        workspace = new_workspace(B, H, N, v.device)
+        workspace.zero_()
+    rc = lib.fp4attn_forward_bf16qk(_ptr(q), _ptr(k), _ptr(v), Shape(B, H, N, D), float(softmax_scale), _ptr(o),
+                                    _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_forward_bf16qk")
     return o, lse
 
 
