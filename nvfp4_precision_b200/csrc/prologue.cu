@@ -58,6 +58,7 @@ struct __align__(1024) ProSmem {
     float inv_scale[128];            // fp32 1 / value of each UE4M3 code (0 for code 0)
     uint64_t bar[NBUF];
     int next_ticket[NBUF];
+    int4 next_tile[NBUF];            // the ticket decoded by thread 0: (kind, head, tile, -)
     int mean_head;
     int abort_flag;
 };
@@ -173,9 +174,10 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
         kind = (smooth ? 0 : 1) + l / Th;
         tile = l % Th;
     };
-    auto issue = [&](int t, int buf) {  // thread 0 only
+    auto issue = [&](int t, int buf) {  // thread 0 only; also publishes the decoded ticket
         int kind, bh, tile;
         decode(t, kind, bh, tile);
+        sm.next_tile[buf] = make_int4(kind, bh, tile, 0);
         const CUtensorMap* map = (kind == KIND_Q) ? &tm_q : &tm_k;
         const uint64_t pol = (kind == KIND_KSUM) ? pol_keep : pol_stream;
         const uint32_t bar = smem_u32(&sm.bar[buf]);
@@ -214,8 +216,8 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
         }
     };
     while (t < total) {
-        int kind, bh, tile;
-        decode(t, kind, bh, tile);
+        const int4 dt = sm.next_tile[buf];  // decoded by thread 0 with the ticket
+        const int kind = dt.x, bh = dt.y, tile = dt.z;
         const bool landed = mbar_wait(smem_u32(&sm.bar[buf]), (phase >> buf) & 1u, &sm.abort_flag, a.status, kSpinLimitNs);
         if (__syncthreads_or(!landed)) break;
         phase ^= 1u << buf;
@@ -242,7 +244,9 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
                 const float v[4] = {bf16lo(kw[rr].x), bf16hi(kw[rr].x), bf16lo(kw[rr].y), bf16hi(kw[rr].y)};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    if (fabsf(v[c]) < kKeyLimit) acc[c] += __float2ll_rn(__fmul_rn(v[c], kTwo24)); else bad = true;
+                    const bool in_range = fabsf(v[c]) < kKeyLimit;
+                    acc[c] += in_range ? __float2ll_rn(__fmul_rn(v[c], kTwo24)) : 0ll;
+                    bad |= !in_range;
                 }
             }
             if (bad) set_status(a.status, FP4ATTN_ERR_RANGE);
