@@ -57,6 +57,8 @@ def lib():
         L.oracle_quantize_qk.restype = ctypes.c_int
         L.oracle_quantize_qk.argtypes = [P, P, i64, i64, i64, ctypes.c_float, ctypes.c_float,
                                          ctypes.c_uint32, P, P, P, P, P]
+        L.oracle_dynamic_gscale.restype = ctypes.c_int
+        L.oracle_dynamic_gscale.argtypes = [P, P, i64, i64, i64, ctypes.c_uint32, P, P]
         L.oracle_dequant.argtypes = [P, P, ctypes.c_float, i64, P]
         L.oracle_attention_head.argtypes = [P, P, P, i64, ctypes.c_double, P, i64, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
@@ -154,15 +156,33 @@ def quantize_rows(y: np.ndarray, g: float = 1.0):
     return codes, scales
 
 
-def quantize_qk(q_bits: np.ndarray, k_bits: np.ndarray, gq: float = 1.0, gk: float = 1.0, flags: int = 0):
-    """Whole prologue on uint16 bf16 bits [B,H,N,128].
-
-    Returns dict(q_codes [B,H,N,64], q_scales [B,H,N,8], k_codes, k_scales,
-    k_mean [B,H,128] float32, status)."""
+def dynamic_gscale(q_bits: np.ndarray, k_bits: np.ndarray, flags: int = 0):
+    """Per-tensor scales from the transformed tensors' largest magnitudes:
+    g = fl32(amax / (6 * 448)), at least 2^-64.  Returns (gq, gk, status) with
+    gq, gk as np.float32."""
     q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
     k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
     B, H, N, D = q_bits.shape
     assert D == 128 and k_bits.shape == q_bits.shape
+    g = np.zeros(2, np.float32)
+    st = lib().oracle_dynamic_gscale(_p(q_bits), _p(k_bits), B, H, N, flags, _p(g[:1]), _p(g[1:]))
+    return g[0], g[1], st
+
+
+def quantize_qk(q_bits: np.ndarray, k_bits: np.ndarray, gq: float = 1.0, gk: float = 1.0, flags: int = 0,
+                dynamic: bool = False):
+    """Whole prologue on uint16 bf16 bits [B,H,N,128].  dynamic=True replaces
+    gq and gk by dynamic_gscale(q_bits, k_bits, flags).
+
+    Returns dict(q_codes [B,H,N,64], q_scales [B,H,N,8], k_codes, k_scales,
+    k_mean [B,H,128] float32, gq, gk (float32), status)."""
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    B, H, N, D = q_bits.shape
+    assert D == 128 and k_bits.shape == q_bits.shape
+    dst = OK
+    if dynamic:
+        gq, gk, dst = dynamic_gscale(q_bits, k_bits, flags)
     out = dict(
         q_codes=np.empty((B, H, N, 64), np.uint8), q_scales=np.empty((B, H, N, 8), np.uint8),
         k_codes=np.empty((B, H, N, 64), np.uint8), k_scales=np.empty((B, H, N, 8), np.uint8),
@@ -170,7 +190,8 @@ def quantize_qk(q_bits: np.ndarray, k_bits: np.ndarray, gq: float = 1.0, gk: flo
     st = lib().oracle_quantize_qk(_p(q_bits), _p(k_bits), B, H, N, gq, gk, flags,
                                   _p(out["q_codes"]), _p(out["q_scales"]),
                                   _p(out["k_codes"]), _p(out["k_scales"]), _p(out["k_mean"]))
-    out["status"] = st
+    out["status"] = st if st != OK else dst
+    out["gq"], out["gk"] = np.float32(gq), np.float32(gk)
     return out
 
 

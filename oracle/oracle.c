@@ -261,6 +261,60 @@ int oracle_quantize_qk(const uint16_t* q, const uint16_t* k, int64_t B, int64_t 
     return err;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Dynamic per-tensor scale.  The page's NVFP4 section ("NVFP4 QAD") names   */
+/* scaling to the largest value as the plain alternative to calibrated       */
+/* static scales; its attention uses a unit scale.  Reading: g maps the      */
+/* largest magnitude of the transformed tensor (all heads, after smoothing   */
+/* and rotation) to the top of the two-level range, 6 (E2M1) x 448 (E4M3):   */
+/* g = fl32(amax / 2688), raised to 2^-64 when smaller (an all-zero tensor   */
+/* included) so that g * scale and 1 / (g * scale) stay finite and normal.   */
+/* ------------------------------------------------------------------------ */
+
+static float tensor_gscale(float amax) {
+    float g = amax / 2688.0f;
+    const float g_min = 5.42101086242752217e-20f; /* 2^-64 */
+    return g < g_min ? g_min : g;
+}
+
+int oracle_dynamic_gscale(const uint16_t* q, const uint16_t* k, int64_t B, int64_t H, int64_t N,
+                          uint32_t flags, float* gq, float* gk) {
+    const int64_t BH = B * H;
+    int err = ORACLE_OK;
+    float* mean = (float*)calloc((size_t)(BH * 128) + 1, sizeof(float));
+    if (!(flags & ORACLE_NO_SMOOTH_K) && N > 0) {
+        int64_t* S = (int64_t*)calloc((size_t)(BH * 128) + 1, sizeof(int64_t));
+        int herr = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic) reduction(max : herr)
+        for (int64_t bh = 0; bh < BH; ++bh) {
+            int e = oracle_ksum(k + bh * N * 128, 1, N, S + bh * 128);
+            if (e > herr) herr = e;
+        }
+        if (herr) err = herr;
+        oracle_kmean(S, BH, N, mean);
+        free(S);
+    }
+    float aq = 0.0f, ak = 0.0f;
+    int rerr = ORACLE_OK;
+#pragma omp parallel for schedule(static) reduction(max : aq, ak, rerr)
+    for (int64_t row = 0; row < BH * N; ++row) {
+        const int64_t bh = row / N;
+        float y[128];
+        if (row_has_nonfinite(q + row * 128) || row_has_nonfinite(k + row * 128)) rerr = ORACLE_ERR_RANGE;
+        transform_row(q + row * 128, NULL, flags, y);
+        for (int i = 0; i < 128; ++i)
+            if (fabsf(y[i]) > aq) aq = fabsf(y[i]);
+        transform_row(k + row * 128, (flags & ORACLE_NO_SMOOTH_K) ? NULL : mean + bh * 128, flags, y);
+        for (int i = 0; i < 128; ++i)
+            if (fabsf(y[i]) > ak) ak = fabsf(y[i]);
+    }
+    if (rerr) err = rerr;
+    free(mean);
+    *gq = tensor_gscale(aq);
+    *gk = tensor_gscale(ak);
+    return err;
+}
+
 void oracle_dequant(const uint8_t* codes, const uint8_t* scales, float g, int64_t rows, float* out) {
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {

@@ -89,6 +89,14 @@ int oracle_quantize_qk(const uint16_t* q, const uint16_t* k, int64_t B, int64_t 
                        uint8_t* q_codes, uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales,
                        float* k_mean);
 
+/* Dynamic per-tensor global scales of Q and K for oracle_quantize_qk: the
+ * largest magnitude of each transformed tensor (smoothing and rotation as
+ * selected by flags, over all B*H heads) mapped to 6 * 448, that is
+ * g = fl32(amax / 2688), raised to 2^-64 when smaller.  Returns ORACLE_OK, or
+ * ORACLE_ERR_RANGE for a non-finite input or |k| >= 2^20 (g then unspecified). */
+int oracle_dynamic_gscale(const uint16_t* q, const uint16_t* k, int64_t B, int64_t H, int64_t N,
+                          uint32_t flags, float* gq, float* gk);
+
 /* Dequantise rows: out = fl(fl(g * dec(scale)) * e2m1(code)). */
 void oracle_dequant(const uint8_t* codes, const uint8_t* scales, float g, int64_t rows, float* out);
 
