@@ -64,12 +64,24 @@ typedef enum {
  * ablation and for checking the quantiser on its own. */
 enum {
     FP4ATTN_NO_SMOOTH_K = 1u,  /* do not subtract the key mean (k_mean reports 0) */
-    FP4ATTN_NO_HADAMARD = 2u   /* do not rotate Q and K                           */
+    FP4ATTN_NO_HADAMARD = 2u,  /* do not rotate Q and K                           */
+    /* fp4attn_quantize_qk_ex only: compute each tensor's global scale from its
+     * largest transformed magnitude instead of taking it from the caller. */
+    FP4ATTN_DYNAMIC_GSCALE = 4u
 };
 
 typedef struct {
     int32_t B, H, N, D;  /* D must be 128; B, H, N >= 0; N <= 262144 */
 } fp4attn_shape;
+
+/* Element strides of a bf16 tensor indexed [b][h][n][c] (c, the 128 channels,
+ * always contiguous).  Each stride must be a positive multiple of 8 elements
+ * (16 bytes) below 2^39; the stride of a dimension of size 1 is ignored.  The
+ * contiguous [B,H,N,128] layout is {H*N*128, N*128, 128}; a [B,N,H,128]
+ * tensor (the layout a QKV projection produces) is {N*H*128, 128, H*128}. */
+typedef struct {
+    int64_t b, h, n;
+} fp4attn_strides;
 
 /* Bytes of workspace that fp4attn_quantize_qk and fp4attn_forward need for
  * this shape (status word, per-head int64 key sums).  Never 0. */
@@ -80,7 +92,8 @@ size_t fp4attn_workspace_bytes(fp4attn_shape s);
  *   q_gscale_dev, k_gscale_dev : device fp32 scalars g (finite, > 0), or NULL
  *     for 1.0.  Block scale s = UE4M3(amax / 6 / g); the value of a code is
  *     g * s * e2m1.
- *   flags : FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD, or 0.
+ *   flags : FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD, or 0 (a dynamic
+ *     global scale needs fp4attn_quantize_qk_ex).
  *   q_codes_dev, k_codes_dev : [B,H,N,64] out.  q_scales_dev, k_scales_dev :
  *     [B,H,N,8] out.  k_mean_dev : [B,H,128] fp32 out, or NULL.
  *   workspace_dev : fp4attn_workspace_bytes(s) bytes; cleared by this call.
@@ -92,6 +105,29 @@ int fp4attn_quantize_qk(const void* q_bf16_dev, const void* k_bf16_dev, fp4attn_
                         uint8_t* q_codes_dev, uint8_t* q_scales_dev,
                         uint8_t* k_codes_dev, uint8_t* k_scales_dev, float* k_mean_dev,
                         void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
+
+/* fp4attn_quantize_qk for Q and K of any strides (fp4attn_strides), with an
+ * optional dynamic global scale.  The codes, scales and k_mean outputs keep the
+ * layouts of fp4attn_quantize_qk.
+ *   flags : as for fp4attn_quantize_qk, plus FP4ATTN_DYNAMIC_GSCALE.
+ *   q_gscale_dev, k_gscale_dev : without FP4ATTN_DYNAMIC_GSCALE, inputs as for
+ *     fp4attn_quantize_qk (NULL for 1.0).  With it, both must be non-NULL and
+ *     receive g = fl32(amax / (6 * 448)), raised to 2^-64 when smaller, where
+ *     amax is the largest magnitude of the whole transformed tensor (after
+ *     smoothing and rotation, over all B*H heads); the block holding that
+ *     value gets scale 448 and code 6.  Pass the same pointers to
+ *     fp4attn_forward.  This reads Q and K twice (two kernel launches).
+ *     Source: FastVideo "Pika H3 Flex in FastVideo", section "NVFP4 QAD"
+ *     (scaling to the largest value, the plain alternative to calibrated
+ *     static scales) and section "FP4 attention" (the per-tensor scale).
+ * Errors as for fp4attn_quantize_qk; FP4ATTN_ERR_INVALID_ARG for a bad stride
+ * or a NULL scale pointer with FP4ATTN_DYNAMIC_GSCALE. */
+int fp4attn_quantize_qk_ex(const void* q_bf16_dev, fp4attn_strides q_strides,
+                           const void* k_bf16_dev, fp4attn_strides k_strides, fp4attn_shape s,
+                           float* q_gscale_dev, float* k_gscale_dev, uint32_t flags,
+                           uint8_t* q_codes_dev, uint8_t* q_scales_dev,
+                           uint8_t* k_codes_dev, uint8_t* k_scales_dev, float* k_mean_dev,
+                           void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
 
 /* Non-causal attention over NVFP4 Q and K and bf16 V (method step 4):
  *   O = softmax(scale * gQ * gK * (Qc K c^T)) V,  Qc, Kc the block-scaled E2M1
@@ -109,6 +145,16 @@ int fp4attn_forward(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
                     void* o_bf16_dev, float* lse_dev,
                     void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
 
+/* fp4attn_forward with V and O of any strides (fp4attn_strides); lse stays
+ * [B,H,N].  O's rows must not overlap one another or any input.  Errors as
+ * for fp4attn_forward; FP4ATTN_ERR_INVALID_ARG for a bad stride. */
+int fp4attn_forward_ex(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
+                       const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                       const float* q_gscale_dev, const float* k_gscale_dev,
+                       const void* v_bf16_dev, fp4attn_strides v_strides, fp4attn_shape s,
+                       float softmax_scale, void* o_bf16_dev, fp4attn_strides o_strides, float* lse_dev,
+                       void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
+
 /* The same non-causal attention with Q and K in BF16 instead of NVFP4: the
  * baseline the FP4 kernel is measured against, and the path for layers kept in
  * BF16 (FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention": two of
@@ -123,6 +169,15 @@ int fp4attn_forward(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
 int fp4attn_forward_bf16qk(const void* q_bf16_dev, const void* k_bf16_dev, const void* v_bf16_dev,
                            fp4attn_shape s, float softmax_scale, void* o_bf16_dev, float* lse_dev,
                            void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
+
+/* fp4attn_forward_bf16qk with Q, K, V and O of any strides (fp4attn_strides);
+ * lse stays [B,H,N].  O's rows must not overlap one another or any input. */
+int fp4attn_forward_bf16qk_ex(const void* q_bf16_dev, fp4attn_strides q_strides,
+                              const void* k_bf16_dev, fp4attn_strides k_strides,
+                              const void* v_bf16_dev, fp4attn_strides v_strides, fp4attn_shape s,
+                              float softmax_scale, void* o_bf16_dev, fp4attn_strides o_strides,
+                              float* lse_dev, void* workspace_dev, size_t workspace_bytes,
+                              cudaStream_t stream);
 
 /* fp4attn_quantize_qk without a workspace argument.  The pages have no
  * counterpart to this entry point: it exists for callers that cannot allocate

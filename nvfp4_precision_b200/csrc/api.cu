@@ -29,6 +29,23 @@ int check_shape(fp4attn_shape s) {
 }
 
 int64_t heads(fp4attn_shape s) { return (int64_t)s.B * s.H; }
+
+// Strides of a [B,H,N,128] bf16 tensor: positive multiples of 8 elements
+// (16 bytes, the tensor-copy rule) below 2^39 elements (2^40 bytes); a
+// dimension of size 1 takes the contiguous stride instead of the caller's.
+bool normalise_strides(fp4attn_shape s, fp4attn_strides in, Strides* out) {
+    const Strides c = contiguous_strides(s.H, s.N);
+    const int64_t v[3] = {s.B == 1 ? c.b : in.b, s.H == 1 ? c.h : in.h, s.N == 1 ? c.n : in.n};
+    for (int64_t x : v)
+        if (x <= 0 || (x & 7) || x >= ((int64_t)1 << 39)) return false;
+    *out = Strides{v[0], v[1], v[2]};
+    return true;
+}
+
+fp4attn_strides contiguous(fp4attn_shape s) {
+    const Strides c = contiguous_strides(s.H, s.N);
+    return fp4attn_strides{c.b, c.h, c.n};
+}
 bool empty(fp4attn_shape s) { return heads(s) == 0 || s.N == 0; }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -92,34 +109,46 @@ size_t fp4attn_workspace_bytes(fp4attn_shape s) {
     return ws_bytes(bh);
 }
 
-int fp4attn_quantize_qk(const void* q, const void* k, fp4attn_shape s, const float* gq,
-                        const float* gk, uint32_t flags, uint8_t* q_codes, uint8_t* q_scales,
-                        uint8_t* k_codes, uint8_t* k_scales, float* k_mean, void* workspace,
-                        size_t workspace_bytes, cudaStream_t stream) {
+int fp4attn_quantize_qk_ex(const void* q, fp4attn_strides q_strides, const void* k, fp4attn_strides k_strides,
+                           fp4attn_shape s, float* gq, float* gk, uint32_t flags, uint8_t* q_codes,
+                           uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales, float* k_mean,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     int st = check_shape(s);
     if (st != FP4ATTN_OK) return st;
-    if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD)) return FP4ATTN_ERR_INVALID_ARG;
+    if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD | FP4ATTN_DYNAMIC_GSCALE))
+        return FP4ATTN_ERR_INVALID_ARG;
+    const bool dynamic = (flags & FP4ATTN_DYNAMIC_GSCALE) != 0;
     if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
         return FP4ATTN_ERR_WORKSPACE;
+    if ((gq && ((uintptr_t)gq & 3)) || (gk && ((uintptr_t)gk & 3))) return FP4ATTN_ERR_INVALID_ARG;
+    if (dynamic && (!gq || !gk)) return FP4ATTN_ERR_INVALID_ARG;
+    Strides qs{}, ks{};
     if (!empty(s)) {
         const void* ptrs[] = {q, k, q_codes, q_scales, k_codes, k_scales};
         for (const void* p : ptrs)
             if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
         if (k_mean && !aligned16(k_mean)) return FP4ATTN_ERR_INVALID_ARG;
-        if ((gq && ((uintptr_t)gq & 3)) || (gk && ((uintptr_t)gk & 3))) return FP4ATTN_ERR_INVALID_ARG;
+        if (!normalise_strides(s, q_strides, &qs) || !normalise_strides(s, k_strides, &ks))
+            return FP4ATTN_ERR_INVALID_ARG;
     }
     cudaError_t e = cudaMemsetAsync(workspace, 0, fp4attn_workspace_bytes(s), stream);
     if (e != cudaSuccess) return launch_status(e);
-    if (empty(s)) return FP4ATTN_OK;
+    if (empty(s)) return dynamic ? launch_status(launch_store_gscales(gq, gk, stream)) : FP4ATTN_OK;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     QuantArgs a;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.k = static_cast<const __nv_bfloat16*>(k);
+    a.qs = qs;
+    a.ks = ks;
     a.BH = (int)heads(s);
+    a.H = s.H;
     a.N = s.N;
-    a.gq = gq;
-    a.gk = gk;
-    a.flags = flags;
+    a.gq = dynamic ? nullptr : gq;
+    a.gk = dynamic ? nullptr : gk;
+    a.g_out[0] = dynamic ? gq : nullptr;
+    a.g_out[1] = dynamic ? gk : nullptr;
+    a.amax = reinterpret_cast<unsigned*>(ws + WS_AMAX_OFFSET);
+    a.flags = (flags & ~(uint32_t)FP4ATTN_DYNAMIC_GSCALE) | (dynamic ? QUANT_DYNAMIC_G : 0u);
     a.q_codes = q_codes;
     a.q_scales = q_scales;
     a.k_codes = k_codes;
@@ -132,10 +161,20 @@ int fp4attn_quantize_qk(const void* q, const void* k, fp4attn_shape s, const flo
     return launch_status(launch_quantize_qk(a, stream));
 }
 
-int fp4attn_forward(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
-                    const uint8_t* k_scales, const float* gq, const float* gk, const void* v,
-                    fp4attn_shape s, float softmax_scale, void* o, float* lse, void* workspace,
-                    size_t workspace_bytes, cudaStream_t stream) {
+int fp4attn_quantize_qk(const void* q, const void* k, fp4attn_shape s, const float* gq, const float* gk,
+                        uint32_t flags, uint8_t* q_codes, uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales,
+                        float* k_mean, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (flags & FP4ATTN_DYNAMIC_GSCALE) return FP4ATTN_ERR_INVALID_ARG;  // its scale pointers are inputs
+    return fp4attn_quantize_qk_ex(q, contiguous(s), k, contiguous(s), s, const_cast<float*>(gq),
+                                  const_cast<float*>(gk), flags, q_codes, q_scales, k_codes, k_scales, k_mean,
+                                  workspace, workspace_bytes, stream);
+}
+
+int fp4attn_forward_ex(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                       const uint8_t* k_scales, const float* gq, const float* gk, const void* v,
+                       fp4attn_strides v_strides, fp4attn_shape s, float softmax_scale, void* o,
+                       fp4attn_strides o_strides, float* lse, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
     int st = check_shape(s);
     if (st != FP4ATTN_OK) return st;
     if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
@@ -147,6 +186,9 @@ int fp4attn_forward(const uint8_t* q_codes, const uint8_t* q_scales, const uint8
         if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
     if (lse && ((uintptr_t)lse & 3)) return FP4ATTN_ERR_INVALID_ARG;
     FwdArgs a;
+    if (!normalise_strides(s, v_strides, &a.vs) || !normalise_strides(s, o_strides, &a.os))
+        return FP4ATTN_ERR_INVALID_ARG;
+    a.H = s.H;
     a.q_codes = q_codes;
     a.q_scales = q_scales;
     a.k_codes = k_codes;
@@ -165,8 +207,18 @@ int fp4attn_forward(const uint8_t* q_codes, const uint8_t* q_scales, const uint8
     return st;
 }
 
-int fp4attn_forward_bf16qk(const void* q, const void* k, const void* v, fp4attn_shape s, float softmax_scale,
-                           void* o, float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int fp4attn_forward(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                    const uint8_t* k_scales, const float* gq, const float* gk, const void* v,
+                    fp4attn_shape s, float softmax_scale, void* o, float* lse, void* workspace,
+                    size_t workspace_bytes, cudaStream_t stream) {
+    return fp4attn_forward_ex(q_codes, q_scales, k_codes, k_scales, gq, gk, v, contiguous(s), s, softmax_scale, o,
+                              contiguous(s), lse, workspace, workspace_bytes, stream);
+}
+
+int fp4attn_forward_bf16qk_ex(const void* q, fp4attn_strides q_strides, const void* k, fp4attn_strides k_strides,
+                              const void* v, fp4attn_strides v_strides, fp4attn_shape s, float softmax_scale,
+                              void* o, fp4attn_strides o_strides, float* lse, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
     int st = check_shape(s);
     if (st != FP4ATTN_OK) return st;
     if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
@@ -178,6 +230,10 @@ int fp4attn_forward_bf16qk(const void* q, const void* k, const void* v, fp4attn_
         if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
     if (lse && ((uintptr_t)lse & 3)) return FP4ATTN_ERR_INVALID_ARG;
     FwdBf16Args a;
+    if (!normalise_strides(s, q_strides, &a.qs) || !normalise_strides(s, k_strides, &a.ks) ||
+        !normalise_strides(s, v_strides, &a.vs) || !normalise_strides(s, o_strides, &a.os))
+        return FP4ATTN_ERR_INVALID_ARG;
+    a.H = s.H;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.k = static_cast<const __nv_bfloat16*>(k);
     a.v = static_cast<const __nv_bfloat16*>(v);
@@ -190,6 +246,12 @@ int fp4attn_forward_bf16qk(const void* q, const void* k, const void* v, fp4attn_
     st = launch_forward_bf16qk(a, stream);
     if (st != FP4ATTN_OK) (void)cudaGetLastError();
     return st;
+}
+
+int fp4attn_forward_bf16qk(const void* q, const void* k, const void* v, fp4attn_shape s, float softmax_scale,
+                           void* o, float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return fp4attn_forward_bf16qk_ex(q, contiguous(s), k, contiguous(s), v, contiguous(s), s, softmax_scale, o,
+                                     contiguous(s), lse, workspace, workspace_bytes, stream);
 }
 
 int fp4attn_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s,

@@ -118,6 +118,8 @@ struct FwdParams {
     const float* gq;
     const float* gk;
     __nv_bfloat16* o;
+    long long o_sb, o_sh, o_sn;  // element strides of O ([B,H,N,128], channels contiguous)
+    int H;
     float* lse;
     int* status;
     uint64_t limit_ns;
@@ -292,6 +294,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         // and its rows are never stored.
         const uint64_t* qs_head = p.q_scales + (size_t)bh * N;
         const uint64_t* ks_head = p.k_scales + (size_t)bh * N;
+        const int v_b = bh / p.H, v_h = bh - v_b * p.H;  // V is addressed as [B][H][N][128]
         const uint32_t qf = smem_u32(&sm.bar_q_full);
 #pragma unroll
         for (int i = 0; i < QT; ++i) {
@@ -327,8 +330,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 const uint32_t full = smem_u32(&sm.bar_kv_full[s]);
                 mbar_arrive_expect_tx(full, K_TILE_BYTES + V_TILE_BYTES);
                 tma_load_3d(smem_u32(sm.kc[s]), &tm_kc, 0, k0, bh, full);
-                tma_load_3d(smem_u32(sm.v[s]), &tm_v, 0, k0, bh, full);
-                tma_load_3d(smem_u32(sm.v[s]) + V_PANEL_BYTES, &tm_v, 64, k0, bh, full);
+                tma_load_4d(smem_u32(sm.v[s]), &tm_v, 0, k0, v_h, v_b, full);
+                tma_load_4d(smem_u32(sm.v[s]) + V_PANEL_BYTES, &tm_v, 64, k0, v_h, v_b, full);
             }
             __syncwarp();
             issued = j + 1;
@@ -577,13 +580,15 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             const float inv_l = 1.0f / l;
             const int n = q0 + BM * qt + row;
             const size_t orow = (size_t)bh * N + n;
+            const int ob = bh / p.H, oh = bh - ob * p.H;
+            __nv_bfloat16* o_row = p.o + ob * p.o_sb + oh * p.o_sh + (long long)n * p.o_sn;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t r[32];
                 tmem_ld32(o_addr + 32u * q, r);
                 tmem_wait_ld();
                 if (n < N) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + 32 * q);
+                    uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * q);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint32_t w[4];
@@ -667,8 +672,8 @@ __global__ void __launch_bounds__(160, 1)
             tma_load_3d(smem_u32(sm.kc), &tm_kc, 0, 0, 0, full);
         } else {
             mbar_arrive_expect_tx(full, 2 * PR_V_PANEL_BYTES);
-            tma_load_3d(smem_u32(sm.v), &tm_v, 0, 0, 0, full);
-            tma_load_3d(smem_u32(sm.v) + PR_V_PANEL_BYTES, &tm_v, 64, 0, 0, full);
+            tma_load_4d(smem_u32(sm.v), &tm_v, 0, 0, 0, 0, full);
+            tma_load_4d(smem_u32(sm.v) + PR_V_PANEL_BYTES, &tm_v, 64, 0, 0, 0, full);
         }
     }
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -757,13 +762,14 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N, uint32_t 
                              strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// V [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x box_rows keys; x is
-// 0 or 64 (0 or 128 bytes), so every box starts on a 16-byte boundary.
-bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N, uint32_t box_rows) {
-    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH};
-    const uint64_t strides[2] = {256, (uint64_t)N * 256};
-    const uint32_t box[3] = {64, box_rows, 1};
-    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(base),
+// V [B][H][N][128 bf16] with element strides st (multiples of 8): 128B-swizzled
+// boxes of 64 channels x box_rows keys of one head; x is 0 or 64 (0 or 128
+// bytes), so every box starts on a 16-byte boundary.
+bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, Strides st, uint32_t box_rows) {
+    const uint64_t dims[4] = {128, (uint64_t)N, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
+    const uint32_t box[4] = {64, box_rows, 1, 1};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(base),
                              dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -776,7 +782,7 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     Maps m;
     if (!make_code_map(&m.qc, a.q_codes, a.BH, a.N, BM) || !make_code_map(&m.kc, a.k_codes, a.BH, a.N, BN) ||
-        !make_v_map(&m.v, a.v, a.BH, a.N, BN))
+        !make_v_map(&m.v, a.v, a.BH / a.H, a.H, a.N, a.vs, BN))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(FwdSmem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = fwd_smem_bytes();
@@ -793,6 +799,10 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     p.gq = a.gq;
     p.gk = a.gk;
     p.o = a.o;
+    p.o_sb = a.os.b;
+    p.o_sh = a.os.h;
+    p.o_sn = a.os.n;
+    p.H = a.H;
     p.lse = a.lse;
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;
@@ -810,7 +820,7 @@ static int launch_probe(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc,
             return FP4ATTN_ERR_CUDA;
         m.v = m.qc;  // unused in this mode
     } else {
-        if (!make_v_map(&m.v, v, 1, 128, 128)) return FP4ATTN_ERR_CUDA;
+        if (!make_v_map(&m.v, v, 1, 1, 128, contiguous_strides(1, 128), 128)) return FP4ATTN_ERR_CUDA;
         m.qc = m.kc = m.v;  // unused in this mode
     }
     const size_t smem = probe_smem_bytes();

@@ -88,6 +88,8 @@ struct Params {
     int n_kt;
     float scale_log2;  // softmax_scale * log2(e)
     __nv_bfloat16* o;
+    long long o_sb, o_sh, o_sn;  // element strides of O ([B,H,N,128], channels contiguous)
+    int H;
     float* lse;
     int* status;
     uint64_t limit_ns;
@@ -171,12 +173,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         // A query tile past N is copied all the same (the copy fills zeros)
         // and its rows are never stored.
         const uint32_t qf = smem_u32(&sm.bar_q_full);
+        const int hb = bh / p.H, hh = bh - hb * p.H;  // Q, K, V are addressed as [B][H][N][128]
         if (lane == 0) {
             mbar_arrive_expect_tx(qf, QT * TILE_BYTES);
 #pragma unroll
             for (int i = 0; i < QT; ++i) {
-                tma_load_3d(smem_u32(sm.q[i]), &tm_q, 0, q0 + BM * i, bh, qf);
-                tma_load_3d(smem_u32(sm.q[i]) + PANEL_BYTES, &tm_q, 64, q0 + BM * i, bh, qf);
+                tma_load_4d(smem_u32(sm.q[i]), &tm_q, 0, q0 + BM * i, hh, hb, qf);
+                tma_load_4d(smem_u32(sm.q[i]) + PANEL_BYTES, &tm_q, 64, q0 + BM * i, hh, hb, qf);
             }
         }
         int issued = 0;
@@ -189,10 +192,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t full = smem_u32(&sm.bar_kv_full[s]);
                 const int k0 = j * BN;
                 mbar_arrive_expect_tx(full, 2 * TILE_BYTES);
-                tma_load_3d(smem_u32(sm.k[s]), &tm_k, 0, k0, bh, full);
-                tma_load_3d(smem_u32(sm.k[s]) + PANEL_BYTES, &tm_k, 64, k0, bh, full);
-                tma_load_3d(smem_u32(sm.v[s]), &tm_v, 0, k0, bh, full);
-                tma_load_3d(smem_u32(sm.v[s]) + PANEL_BYTES, &tm_v, 64, k0, bh, full);
+                tma_load_4d(smem_u32(sm.k[s]), &tm_k, 0, k0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.k[s]) + PANEL_BYTES, &tm_k, 64, k0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.v[s]), &tm_v, 0, k0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.v[s]) + PANEL_BYTES, &tm_v, 64, k0, hh, hb, full);
             }
             __syncwarp();
             issued = j + 1;
@@ -388,13 +391,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float inv_l = 1.0f / l;
             const int n = q0 + BM * qt + row;
             const size_t orow = (size_t)bh * N + n;
+            const int ob = bh / p.H, oh = bh - ob * p.H;
+            __nv_bfloat16* o_row = p.o + ob * p.o_sb + oh * p.o_sh + (long long)n * p.o_sn;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t r[32];
                 tmem_ld32(o_addr + 32u * q, r);
                 tmem_wait_ld();
                 if (n < N) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow * 128 + 32 * q);
+                    uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * q);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint32_t w[4];
@@ -419,13 +424,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
-// [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x 128 rows; x is 0 or 64
-// (0 or 128 bytes), so every box starts on a 16-byte boundary.
-bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N) {
-    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH};
-    const uint64_t strides[2] = {256, (uint64_t)N * 256};
-    const uint32_t box[3] = {64, 128, 1};
-    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(base), dims,
+// [B][H][N][128 bf16] with element strides st (multiples of 8): 128B-swizzled
+// boxes of 64 channels x 128 rows of one head; x is 0 or 64 (0 or 128 bytes),
+// so every box starts on a 16-byte boundary.
+bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, Strides st) {
+    const uint64_t dims[4] = {128, (uint64_t)N, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(base), dims,
                              strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -434,8 +440,9 @@ bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N) {
 int launch_forward_bf16qk(const FwdBf16Args& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     CUtensorMap tq, tk, tv;
-    if (!make_rows_map(&tq, a.q, a.BH, a.N) || !make_rows_map(&tk, a.k, a.BH, a.N) ||
-        !make_rows_map(&tv, a.v, a.BH, a.N))
+    const int B = a.BH / a.H;
+    if (!make_rows_map(&tq, a.q, B, a.H, a.N, a.qs) || !make_rows_map(&tk, a.k, B, a.H, a.N, a.ks) ||
+        !make_rows_map(&tv, a.v, B, a.H, a.N, a.vs))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = sizeof(Smem) + 1024;
@@ -448,6 +455,10 @@ int launch_forward_bf16qk(const FwdBf16Args& a, cudaStream_t stream) {
     const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 0.08838834764831845f;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.o = a.o;
+    p.o_sb = a.os.b;
+    p.o_sh = a.os.h;
+    p.o_sn = a.os.n;
+    p.H = a.H;
     p.lse = a.lse;
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;

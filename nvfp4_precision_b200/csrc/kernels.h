@@ -9,11 +9,14 @@ namespace fp4attn {
 
 constexpr int D = 128;
 
-// Workspace layout: [0,4) status word, [64,68) prologue tile ticket counter,
-// rest of [0,256) spare; [256, 256 + 8*BH*128) int64 key column sums; then
-// one uint32 per head (key-sum tiles completed).
+// Workspace layout: [0,4) status word, [64,68) and [68,72) tile ticket
+// counters of the two prologue launches, [128,136) fp32 bit patterns of the
+// transformed amax of Q and K (dynamic global scales), rest of [0,256) spare;
+// [256, 256 + 8*BH*128) int64 key column sums; then one uint32 per head
+// (key-sum tiles completed).
 constexpr size_t WS_STATUS_BYTES = 256;
 constexpr size_t WS_TICKET_OFFSET = 64;
+constexpr size_t WS_AMAX_OFFSET = 128;
 inline size_t ws_ksum_offset() { return WS_STATUS_BYTES; }
 inline size_t ws_counter_offset(int64_t BH) { return WS_STATUS_BYTES + (size_t)BH * D * 8; }
 inline size_t ws_bytes(int64_t BH) {
@@ -21,12 +24,26 @@ inline size_t ws_bytes(int64_t BH) {
     return (b + 255) / 256 * 256;
 }
 
+// Element strides of a [B,H,N,128] bf16 tensor (the channel stride is 1).
+struct Strides {
+    int64_t b, h, n;
+};
+inline Strides contiguous_strides(int H, int N) {
+    return Strides{(int64_t)H * N * D, (int64_t)N * D, (int64_t)D};
+}
+
+// Flag of QuantArgs: compute g of Q and K from the transformed amax.
+constexpr uint32_t QUANT_DYNAMIC_G = 4u;
+
 struct QuantArgs {
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
-    int BH, N;
-    const float* gq;  // device scalar or nullptr (1.0)
+    Strides qs, ks;
+    int BH, H, N;
+    const float* gq;  // device scalar or nullptr (1.0); ignored with QUANT_DYNAMIC_G
     const float* gk;
+    float* g_out[2];  // QUANT_DYNAMIC_G: receive the computed g of Q and K
+    unsigned* amax;   // QUANT_DYNAMIC_G: two zeroed words (fp32 bits of the amax)
     uint32_t flags;
     uint8_t* q_codes;
     uint8_t* q_scales;
@@ -40,6 +57,8 @@ struct QuantArgs {
 };
 
 cudaError_t launch_quantize_qk(const QuantArgs& a, cudaStream_t stream);
+// Dynamic global scales of empty tensors (amax 0): store the smallest g, 2^-64.
+cudaError_t launch_store_gscales(float* gq, float* gk, cudaStream_t stream);
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
                            float* out, cudaStream_t stream);
@@ -60,7 +79,8 @@ struct FwdArgs {
     const float* gq;
     const float* gk;
     const __nv_bfloat16* v;
-    int BH, N;
+    Strides vs, os;
+    int BH, H, N;
     float softmax_scale;
     __nv_bfloat16* o;
     float* lse;
@@ -71,7 +91,8 @@ struct FwdBf16Args {
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
-    int BH, N;
+    Strides qs, ks, vs, os;
+    int BH, H, N;
     float softmax_scale;
     __nv_bfloat16* o;
     float* lse;

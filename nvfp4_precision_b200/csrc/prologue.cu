@@ -19,7 +19,13 @@
 //                  E2M1 codes of y * (1/(g*scale)).
 // The Q tiles of a head sit between its key-sum and K tiles, so the second
 // read of K mostly hits L2 (key-sum loads are marked evict-last, the others
-// evict-first).  Tiles arrive by TMA (128B swizzle) in a ring of NBUF buffers
+// evict-first).  Q and K may have any [B,H,N,128] strides (a 4-D tensor map).
+//
+// Dynamic global scales (g = amax / (6*448) of each whole transformed tensor)
+// take two launches of the same kernel: the first (AMAX) does the key sums and
+// the transform of every Q and K row and reduces the largest magnitude of each
+// tensor into two workspace words; the second encodes, with g computed from
+// those words, and skips the key sums, which are already complete.  Tiles arrive by TMA (128B swizzle) in a ring of NBUF buffers
 // per CTA.  Each tile is first copied from its buffer into registers; after
 // one barrier the buffer is refilled with the tile NBUF tickets ahead, so every
 // buffer is in flight while a tile is computed.
@@ -67,14 +73,23 @@ struct ProArgs {
     uint8_t* codes[2];
     uint8_t* scales[2];
     const float* g[2];
+    float* g_out[2];   // encode launch of the dynamic path: receive g of Q and K
+    unsigned* amax;    // dynamic path: fp32 bits of the transformed amax of Q and K
     long long* ksum;
     unsigned* head_ready;
     unsigned* ticket;
     float* k_mean;
-    int BH, N, n_tiles;
+    int BH, H, N, n_tiles;
     uint32_t flags;
+    bool sums_ready;   // the key sums of every head are complete: no key-sum tiles
     int* status;
 };
+
+// g = fl32(amax / (6*448)), raised to 2^-64 when smaller, so that g * scale
+// and its reciprocal stay finite and normal.
+__device__ __forceinline__ float tensor_gscale(float amax) {
+    return fmaxf(__fdiv_rn(amax, 2688.0f), 5.42101086242752217e-20f);
+}
 
 __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
@@ -91,12 +106,12 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
-__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
-                                                 int32_t c2, uint32_t bar, uint64_t policy) {
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                 int32_t c2, int32_t c3, uint32_t bar, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
-        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(policy)
         : "memory");
 }
 
@@ -135,6 +150,9 @@ __device__ __forceinline__ void block_scale(float a, float g, bool g_is_one, con
     }
 }
 
+// AMAX = true: the first launch of the dynamic-scale path (key sums and the
+// transformed amax of Q and K; no codes are written).
+template <bool AMAX>
 __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                const __grid_constant__ CUtensorMap tm_k,
                                                                const ProArgs a) {
@@ -145,7 +163,8 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
     const int Th = a.n_tiles;
     const bool smooth = !(a.flags & FP4ATTN_NO_SMOOTH_K);
     const bool hadamard = !(a.flags & FP4ATTN_NO_HADAMARD);
-    const int per_head = (smooth ? 3 : 2) * Th;
+    const int first_kind = (smooth && !a.sums_ready) ? KIND_KSUM : KIND_Q;
+    const int per_head = (3 - first_kind) * Th;
     const int total = a.BH * per_head;
 
     if (tid == 0) {
@@ -161,8 +180,17 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
         sm.inv_scale[tid] = (sd != 0.0f) ? __frcp_rn(sd) : 0.0f;
     }
     float gq = 1.0f, gk = 1.0f;
-    if (a.g[0]) gq = *a.g[0];
-    if (a.g[1]) gk = *a.g[1];
+    if (!AMAX && a.amax) {  // encode launch of the dynamic path
+        gq = tensor_gscale(__uint_as_float(__ldcg(a.amax)));
+        gk = tensor_gscale(__uint_as_float(__ldcg(a.amax + 1)));
+        if (blockIdx.x == 0 && tid == 0) {
+            if (a.g_out[0]) *a.g_out[0] = gq;
+            if (a.g_out[1]) *a.g_out[1] = gk;
+        }
+    } else if (!AMAX) {
+        if (a.g[0]) gq = *a.g[0];
+        if (a.g[1]) gk = *a.g[1];
+    }
     if (tid == 0 && !(gq > 0.0f && gq < INFINITY && gk > 0.0f && gk < INFINITY)) set_status(a.status, FP4ATTN_ERR_RANGE);
     __syncthreads();
 
@@ -171,7 +199,7 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
     auto decode = [&](int t, int& kind, int& bh, int& tile) {
         bh = t / per_head;
         const int l = t - bh * per_head;
-        kind = (smooth ? 0 : 1) + l / Th;
+        kind = first_kind + l / Th;
         tile = l % Th;
     };
     auto issue = [&](int t, int buf) {  // thread 0 only; also publishes the decoded ticket
@@ -181,12 +209,14 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
         const CUtensorMap* map = (kind == KIND_Q) ? &tm_q : &tm_k;
         const uint64_t pol = (kind == KIND_KSUM) ? pol_keep : pol_stream;
         const uint32_t bar = smem_u32(&sm.bar[buf]);
+        const int b = bh / a.H, h = bh - b * a.H;
         mbar_arrive_expect_tx(bar, TILE_BYTES);
-        tma_load_3d_hint(smem_u32(sm.tile[buf]), map, 0, tile * 128, bh, bar, pol);
-        tma_load_3d_hint(smem_u32(sm.tile[buf]) + HALF_BYTES, map, 64, tile * 128, bh, bar, pol);
+        tma_load_4d_hint(smem_u32(sm.tile[buf]), map, 0, tile * 128, h, b, bar, pol);
+        tma_load_4d_hint(smem_u32(sm.tile[buf]) + HALF_BYTES, map, 64, tile * 128, h, b, bar, pol);
     };
 
     uint32_t in_flight = 0u;  // bit b: a copy into buffer b is outstanding (thread 0, which issues them)
+    float amax_q = 0.0f, amax_k = 0.0f;  // AMAX: largest |y| of this thread's valid Q and K rows
     if (tid == 0) {
         for (int b = 0; b < NBUF; ++b) {
             const int tk = (int)atomicAdd(a.ticket, 1u);
@@ -386,13 +416,22 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
                 for (int k = 0; k < 32; ++k) P[k] = __fmul2_rn(P[k], f2(c, c));
             }
 
+            const bool valid = (tile * 128 + r) < N;
+            if (!finite && valid) set_status(a.status, FP4ATTN_ERR_RANGE);
+            if constexpr (AMAX) {
+                // rows past N hold the copy's zero fill (minus the mean for K): skip them
+                if (valid) {
+                    float m = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) m = fmax3(m, fabsf(P[k].x), fabsf(P[k].y));
+                    if (which) amax_k = fmaxf(amax_k, m); else amax_q = fmaxf(amax_q, m);
+                }
+            } else {
             // NVFP4 pack.  This lane holds blocks 2h, 2h+1 (the .x lanes of
             // P[0..15], P[16..31]) and 4+2h, 5+2h (the .y lanes); block b's codes
             // are bytes 8b..8b+7 of the row.
             const float gw = which ? gk : gq;
             const bool g_is_one = (gw == 1.0f);
-            const bool valid = (tile * 128 + r) < N;
-            if (!finite && valid) set_status(a.status, FP4ATTN_ERR_RANGE);
             const size_t row = (size_t)bh * N + (size_t)tile * 128 + r;
             uint32_t s_b[4];  // scale bytes of blocks 2h, 2h+1, 4+2h, 5+2h
             uint32_t w_lo[4], w_hi[4];
@@ -421,10 +460,20 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
                 dst[2 + h] = make_uint4(w_hi[0], w_hi[1], w_hi[2], w_hi[3]);
                 *reinterpret_cast<uint32_t*>((which ? a.scales[1] : a.scales[0]) + row * 8 + 4 * h) = sword;
             }
+            }  // pack
         }
         // the next buffer's ticket was written at least one barrier ago
         buf = (buf + 1) % NBUF;
         t = sm.next_ticket[buf];
+    }
+    if constexpr (AMAX) {
+        // magnitudes are >= 0, so their fp32 bit patterns order like the values
+        const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_q));
+        const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_k));
+        if ((tid & 31) == 0) {
+            if (wq) atomicMax(a.amax, wq);
+            if (wk) atomicMax(a.amax + 1, wk);
+        }
     }
     // wind down after an abort: let this CTA's own copies land before exiting
     if (tid == 0) {
@@ -436,32 +485,55 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
 
 size_t pro_smem_bytes() { return sizeof(ProSmem) + 1024; }
 
-bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int BH, int N) {
-    // [BH][N][128 bf16]: 128B-swizzled boxes of 64 channels x 128 rows; x is 0 or 64
-    // (0 or 128 bytes), so every box starts on a 16-byte boundary.
-    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH};
-    const uint64_t strides[2] = {256, (uint64_t)N * 256};
-    const uint32_t box[3] = {64, 128, 1};
-    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(base), dims,
+// [B][H][N][128 bf16] with element strides st: 128B-swizzled boxes of 64
+// channels x 128 rows of one head; x is 0 or 64 (0 or 128 bytes), so every box
+// starts on a 16-byte boundary.  The strides must be multiples of 8 elements.
+bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, Strides st) {
+    const uint64_t dims[4] = {128, (uint64_t)N, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(base), dims,
                              strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-}  // namespace
-
-cudaError_t launch_quantize_qk(const QuantArgs& q, cudaStream_t stream) {
-    if (q.BH == 0 || q.N == 0) return cudaSuccess;
-    CUtensorMap tm_q, tm_k;
-    if (!make_rows_map(&tm_q, q.q, q.BH, q.N) || !make_rows_map(&tm_k, q.k, q.BH, q.N)) return cudaErrorInvalidValue;
+template <bool AMAX>
+cudaError_t launch_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ProArgs& a, cudaStream_t stream) {
     static_assert(sizeof(ProSmem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = pro_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(prologue_kernel<AMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prologue_kernel, PRO_THREADS, smem)) !=
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prologue_kernel<AMAX>, PRO_THREADS, smem)) !=
         cudaSuccess)
         return e;
+    const bool sum_tiles = !(a.flags & FP4ATTN_NO_SMOOTH_K) && !a.sums_ready;
+    const long long tiles = (long long)a.BH * a.n_tiles * (sum_tiles ? 3 : 2);
+    long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
+    if (grid > tiles) grid = tiles;
+    prologue_kernel<AMAX><<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, a);
+    return cudaGetLastError();
+}
+
+__global__ void store_gscales_kernel(float* gq, float* gk) {
+    *gq = tensor_gscale(0.0f);
+    *gk = tensor_gscale(0.0f);
+}
+
+}  // namespace
+
+cudaError_t launch_store_gscales(float* gq, float* gk, cudaStream_t stream) {
+    store_gscales_kernel<<<1, 1, 0, stream>>>(gq, gk);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_qk(const QuantArgs& q, cudaStream_t stream) {
+    if (q.BH == 0 || q.N == 0) return cudaSuccess;
+    const int B = q.BH / q.H;
+    CUtensorMap tm_q, tm_k;
+    if (!make_rows_map(&tm_q, q.q, B, q.H, q.N, q.qs) || !make_rows_map(&tm_k, q.k, B, q.H, q.N, q.ks))
+        return cudaErrorInvalidValue;
     ProArgs a{};
     a.codes[0] = q.q_codes;
     a.codes[1] = q.k_codes;
@@ -474,15 +546,24 @@ cudaError_t launch_quantize_qk(const QuantArgs& q, cudaStream_t stream) {
     a.ticket = q.ticket;
     a.k_mean = q.k_mean;
     a.BH = q.BH;
+    a.H = q.H;
     a.N = q.N;
     a.n_tiles = (q.N + 127) / 128;
-    a.flags = q.flags;
+    a.flags = q.flags & ~QUANT_DYNAMIC_G;
     a.status = q.status;
-    const long long tiles = (long long)a.BH * a.n_tiles * ((q.flags & FP4ATTN_NO_SMOOTH_K) ? 2 : 3);
-    long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
-    if (grid > tiles) grid = tiles;
-    prologue_kernel<<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, a);
-    return cudaGetLastError();
+    if (!(q.flags & QUANT_DYNAMIC_G)) return launch_pass<false>(tm_q, tm_k, a, stream);
+    // dynamic global scales: amax pass (with the key sums), then the encode pass
+    ProArgs m = a;
+    m.amax = q.amax;
+    m.k_mean = nullptr;
+    cudaError_t e = launch_pass<true>(tm_q, tm_k, m, stream);
+    if (e != cudaSuccess) return e;
+    a.amax = q.amax;
+    a.g_out[0] = q.g_out[0];
+    a.g_out[1] = q.g_out[1];
+    a.ticket = q.ticket + 1;
+    a.sums_ready = true;
+    return launch_pass<false>(tm_q, tm_k, a, stream);
 }
 
 }  // namespace fp4attn

@@ -25,10 +25,11 @@ ERR_TIMEOUT = 5
 ERR_WORKSPACE = 6
 NO_SMOOTH_K = 1
 NO_HADAMARD = 2
+DYNAMIC_GSCALE = 4
 
 EXPORTS = (
-    "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_quantize_qk_noalloc", "fp4attn_forward",
-    "fp4attn_forward_bf16qk",
+    "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_quantize_qk_ex", "fp4attn_quantize_qk_noalloc",
+    "fp4attn_forward", "fp4attn_forward_ex", "fp4attn_forward_bf16qk", "fp4attn_forward_bf16qk_ex",
     "fp4attn_dequant",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
@@ -37,6 +38,11 @@ EXPORTS = (
 
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("D", ctypes.c_int32)]
+
+
+class Strides(ctypes.Structure):
+    """Element strides (b, h, n) of a [B,H,N,128] tensor whose channels are contiguous."""
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("n", ctypes.c_int64)]
 
 
 class Fp4AttnError(RuntimeError):
@@ -55,6 +61,15 @@ def _load():
     L.fp4attn_workspace_bytes.argtypes = [Shape]
     L.fp4attn_quantize_qk.restype = ctypes.c_int
     L.fp4attn_quantize_qk.argtypes = [P, P, Shape, P, P, U32, P, P, P, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_quantize_qk_ex.restype = ctypes.c_int
+    L.fp4attn_quantize_qk_ex.argtypes = [P, Strides, P, Strides, Shape, P, P, U32, P, P, P, P, P, P,
+                                         ctypes.c_size_t, P]
+    L.fp4attn_forward_ex.restype = ctypes.c_int
+    L.fp4attn_forward_ex.argtypes = [P, P, P, P, P, P, P, Strides, Shape, ctypes.c_float, P, Strides, P, P,
+                                     ctypes.c_size_t, P]
+    L.fp4attn_forward_bf16qk_ex.restype = ctypes.c_int
+    L.fp4attn_forward_bf16qk_ex.argtypes = [P, Strides, P, Strides, P, Strides, Shape, ctypes.c_float, P, Strides,
+                                            P, P, ctypes.c_size_t, P]
     L.fp4attn_quantize_qk_noalloc.restype = ctypes.c_int
     L.fp4attn_quantize_qk_noalloc.argtypes = [P, P, Shape, P, P, U32, P, P, P, P, P, P, P]
     L.fp4attn_forward.restype = ctypes.c_int
@@ -107,6 +122,14 @@ def shape_of(t: torch.Tensor) -> Shape:
     return Shape(B, H, N, D)
 
 
+def strides_of(t: torch.Tensor) -> Strides:
+    """Strides of a [B,H,N,128] tensor or view (e.g. ``x.transpose(1, 2)`` of a
+    [B,N,H,128] tensor); the channels must be contiguous.  The library checks
+    the rest (positive multiples of 8)."""
+    assert t.dim() == 4 and t.stride(3) == 1, "the channel dimension must be contiguous"
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
 def fp4attn_workspace_bytes(B: int, H: int, N: int, D: int = 128) -> int:
     return int(lib.fp4attn_workspace_bytes(Shape(B, H, N, D)))
 
@@ -118,12 +141,17 @@ def new_workspace(B: int, H: int, N: int, device="cuda") -> torch.Tensor:
 
 def fp4attn_quantize_qk(q: torch.Tensor, k: torch.Tensor, q_gscale: Optional[torch.Tensor] = None,
                         k_gscale: Optional[torch.Tensor] = None, flags: int = 0, out: Optional[dict] = None,
-                        k_mean: bool = True, workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
-    """Smooth K + Hadamard + NVFP4 pack of bf16 [B,H,N,128] Q and K.
+                        k_mean: bool = True, workspace: Optional[torch.Tensor] = None, stream=None,
+                        dynamic_gscale: bool = False) -> dict:
+    """Smooth K + Hadamard + NVFP4 pack of bf16 [B,H,N,128] Q and K (any
+    strides with contiguous channels).  dynamic_gscale=True computes each
+    tensor's global scale from its transformed amax into q_gscale / k_gscale
+    (allocated when None) instead of reading them.
 
-    Returns dict(q_codes, q_scales, k_codes, k_scales, k_mean, workspace)."""
+    Returns dict(q_codes, q_scales, k_codes, k_scales, k_mean, workspace) and,
+    with dynamic_gscale, q_gscale and k_gscale (fp32 device scalars to pass to
+    fp4attn_forward)."""
     assert q.dtype == torch.bfloat16 and k.dtype == torch.bfloat16 and q.shape == k.shape
-    assert q.is_contiguous() and k.is_contiguous()
     B, H, N, D = q.shape
     dev = q.device
     if out is None:
@@ -134,12 +162,18 @@ def fp4attn_quantize_qk(q: torch.Tensor, k: torch.Tensor, q_gscale: Optional[tor
                    k_mean=torch.empty((B, H, 128), dtype=torch.float32, device=dev) if k_mean else None)
     if workspace is None:
         workspace = new_workspace(B, H, N, dev)
-    rc = lib.fp4attn_quantize_qk(_ptr(q), _ptr(k), Shape(B, H, N, D), _ptr(q_gscale), _ptr(k_gscale),
-                                 int(flags), _ptr(out["q_codes"]), _ptr(out["q_scales"]), _ptr(out["k_codes"]),
-                                 _ptr(out["k_scales"]), _ptr(out.get("k_mean")), _ptr(workspace),
-                                 workspace.numel(), _stream(stream))
-    _check(rc, "fp4attn_quantize_qk")
+    if dynamic_gscale:
+        flags = int(flags) | DYNAMIC_GSCALE
+        q_gscale = torch.empty(1, dtype=torch.float32, device=dev) if q_gscale is None else q_gscale
+        k_gscale = torch.empty(1, dtype=torch.float32, device=dev) if k_gscale is None else k_gscale
+    rc = lib.fp4attn_quantize_qk_ex(_ptr(q), strides_of(q), _ptr(k), strides_of(k), Shape(B, H, N, D),
+                                    _ptr(q_gscale), _ptr(k_gscale), int(flags), _ptr(out["q_codes"]),
+                                    _ptr(out["q_scales"]), _ptr(out["k_codes"]), _ptr(out["k_scales"]),
+                                    _ptr(out.get("k_mean")), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_quantize_qk_ex")
     out["workspace"] = workspace
+    if dynamic_gscale:
+        out["q_gscale"], out["k_gscale"] = q_gscale, k_gscale
     return out
 
 
@@ -173,41 +207,48 @@ def fp4attn_quantize_qk_noalloc(q: torch.Tensor, k: torch.Tensor, q_gscale: Opti
 def fp4attn_forward(q_codes, q_scales, k_codes, k_scales, v: torch.Tensor, q_gscale=None, k_gscale=None,
                     softmax_scale: float = 0.0, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                     want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
-    """Non-causal attention over NVFP4 Q/K and bf16 V.  Returns (O, lse or None)."""
-    assert v.dtype == torch.bfloat16 and v.is_contiguous()
+    """Non-causal attention over NVFP4 Q/K and bf16 V [B,H,N,128] (any strides
+    with contiguous channels; so may a caller-supplied O be).  Returns
+    (O, lse or None); a new O is contiguous [B,H,N,128]."""
+    assert v.dtype == torch.bfloat16
     B, H, N, D = v.shape
     if o is None:
-        o = torch.empty_like(v)
+        o = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=v.device)
+    assert o.shape == v.shape and o.dtype == torch.bfloat16
     if want_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
     if workspace is None:
         workspace = new_workspace(B, H, N, v.device)
         workspace.zero_()
-    rc = lib.fp4attn_forward(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(q_gscale),
-                             _ptr(k_gscale), _ptr(v), Shape(B, H, N, D), float(softmax_scale), _ptr(o), _ptr(lse),
-                             _ptr(workspace), workspace.numel(), _stream(stream))
-    _check(rc, "fp4attn_forward")
+    rc = lib.fp4attn_forward_ex(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(q_gscale),
+                                _ptr(k_gscale), _ptr(v), strides_of(v), Shape(B, H, N, D), float(softmax_scale),
+                                _ptr(o), strides_of(o), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                _stream(stream))
+    _check(rc, "fp4attn_forward_ex")
     return o, lse
 
 
 def fp4attn_forward_bf16qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float = 0.0,
                            o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                            want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
-    """Non-causal attention with bf16 Q, K, V [B,H,N,128] (no quantisation): the
-    BF16 counterpart of fp4attn_forward.  Returns (O, lse or None)."""
+    """Non-causal attention with bf16 Q, K, V [B,H,N,128] (no quantisation; any
+    strides with contiguous channels): the BF16 counterpart of fp4attn_forward.
+    Returns (O, lse or None); a new O is contiguous [B,H,N,128]."""
     for t in (q, k, v):
-        assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == v.shape
+        assert t.dtype == torch.bfloat16 and t.shape == v.shape
     B, H, N, D = v.shape
     if o is None:
-        o = torch.empty_like(v)
+        o = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=v.device)
+    assert o.shape == v.shape and o.dtype == torch.bfloat16
     if want_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
     if workspace is None:
         workspace = new_workspace(B, H, N, v.device)
         workspace.zero_()
-    rc = lib.fp4attn_forward_bf16qk(_ptr(q), _ptr(k), _ptr(v), Shape(B, H, N, D), float(softmax_scale), _ptr(o),
-                                    _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream))
-    _check(rc, "fp4attn_forward_bf16qk")
+    rc = lib.fp4attn_forward_bf16qk_ex(_ptr(q), strides_of(q), _ptr(k), strides_of(k), _ptr(v), strides_of(v),
+                                       Shape(B, H, N, D), float(softmax_scale), _ptr(o), strides_of(o), _ptr(lse),
+                                       _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_forward_bf16qk_ex")
     return o, lse
 
 

@@ -79,3 +79,34 @@ def test_probe_validation(fa):
     assert fa.lib.fp4attn_probe_qk_tile(None, None, None, None, None, None) == fa.ERR_INVALID_ARG
     assert fa.lib.fp4attn_probe_wait_timeout(None, 1000, None) == fa.ERR_INVALID_ARG
     assert fa.lib.fp4attn_encode_f32(None, 5, None, None, None) == fa.ERR_INVALID_ARG
+
+
+def test_strided_and_dynamic_validation_before_launch(fa):
+    """The strided entry points reject bad strides (not a positive multiple of 8
+    elements, or 2^39 and above) and the dynamic scale without its outputs."""
+    S, St = fa.Shape, fa.Strides
+    p = ctypes.c_void_p(4096)
+    ws = ctypes.c_void_p(256)
+    shape = S(2, 3, 128, 128)
+    good = St(3 * 128 * 128, 128 * 128, 128)
+
+    def qex(qs, ks=good, flags=0, g=p):
+        return fa.lib.fp4attn_quantize_qk_ex(p, qs, p, ks, shape, g, g, flags, p, p, p, p, None, ws, 1 << 20, None)
+
+    for bad in (St(3 * 128 * 128, 128 * 128, 100), St(0, 128 * 128, 128), St(-8, 128 * 128, 128),
+                St(3 * 128 * 128, 1 << 39, 128)):
+        assert qex(bad) == fa.ERR_INVALID_ARG
+        assert qex(good, ks=bad) == fa.ERR_INVALID_ARG
+    assert qex(good, flags=fa.DYNAMIC_GSCALE, g=None) == fa.ERR_INVALID_ARG
+    assert qex(good, flags=8) == fa.ERR_INVALID_ARG
+    # the plain entry point takes its scales as inputs: no dynamic scale there
+    assert _q(fa, S(1, 1, 128, 128), flags=fa.DYNAMIC_GSCALE) == fa.ERR_INVALID_ARG
+    bad = St(3 * 128 * 128, 128 * 128, 12)
+    fex = fa.lib.fp4attn_forward_ex
+    assert fex(p, p, p, p, None, None, p, bad, shape, 0.0, p, good, None, p, 1 << 20, None) == fa.ERR_INVALID_ARG
+    assert fex(p, p, p, p, None, None, p, good, shape, 0.0, p, bad, None, p, 1 << 20, None) == fa.ERR_INVALID_ARG
+    bex = fa.lib.fp4attn_forward_bf16qk_ex
+    for i in range(4):
+        st = [good] * 4
+        st[i] = bad
+        assert bex(p, st[0], p, st[1], p, st[2], shape, 0.0, p, st[3], None, p, 1 << 20, None) == fa.ERR_INVALID_ARG
