@@ -44,10 +44,10 @@ PROLOGUE_BYTES_PER_ELEMENT = 5.125  # Q,K bf16 read (2+2) + codes (0.5+0.5) + sc
 # kernel source they were measured on and the workload; a changed kernel reports
 # null until it is profiled again (profiles/ holds the commands).
 ATTN_TRAFFIC_BYTES = {
-    ("a6a1dd35d211ef39", "clip15s"): 2.40e9 + 1.39e9,
+    ("3c2dd89ee5583f05", "clip15s"): 2.450e9 + 1.393e9,
 }
 PROLOGUE_TRAFFIC_BYTES = {
-    ("1eeb4d396cdc574e", "clip15s"): 2.70e9 + 0.725e9,
+    ("2cfa9c01d2643c07", "clip15s"): 2.703e9 + 0.725e9,
 }
 
 
@@ -337,6 +337,49 @@ def run_ours(args, rank, world, local):
                   "fp4_speedup": ms_b / ms_att_max}
         del o2
 
+    # ---- general forms (outside the timed step): the dynamic global scale and
+    # the [B,N,H,128] layout a QKV projection writes ----
+    general = None
+    if not args.no_general:
+        reps = max(2, min(args.steps, 3))
+        gq = torch.empty(1, dtype=torch.float32, device=dev)
+        gk = torch.empty(1, dtype=torch.float32, device=dev)
+
+        def dyn():
+            fa.fp4attn_quantize_qk(q, k, gq, gk, out=out, workspace=ws, stream=stream, dynamic_gscale=True)
+
+        dyn()
+        dev_ = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for e in dev_:
+            e[0].record(stream)
+            dyn()
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms_dyn = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in dev_), world, dev)
+        qt, kt, vt = (x.transpose(1, 2).contiguous().transpose(1, 2) for x in (q, k, v))
+        ot = torch.empty((B, N, H, 128), dtype=torch.bfloat16, device=dev).transpose(1, 2)
+
+        def bnhd_step():
+            fa.fp4attn_quantize_qk(qt, kt, flags=0, out=out, workspace=ws, stream=stream)
+            fa.fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], vt, o=ot,
+                               workspace=ws, stream=stream)
+
+        bnhd_step()
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for e in tev:
+            e[0].record(stream)
+            bnhd_step()
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        st = fa.fp4attn_read_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status after the general forms: {fa.status_string(st)}")
+        ms_t = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in tev), world, dev)
+        general = {"quantize_dynamic_g_ms": ms_dyn,
+                   "quantize_dynamic_g_gbs": pro_bytes / (ms_dyn * 1e-3) / 1e9,
+                   "bnhd_layout_step_ms": ms_t, "bnhd_layout_tflops": F / (ms_t * 1e-3) / 1e12}
+        del qt, kt, vt, ot
+
     csrc = os.path.join(ROOT, "nvfp4_precision_b200", "csrc")
     traffic = ATTN_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "attention.cu")), args.workload))
     pro_traffic = PROLOGUE_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "prologue.cu")), args.workload))
@@ -386,6 +429,7 @@ def run_ours(args, rank, world, local):
             "quantize": {"ms": ms_pro_max, "gbs": pro_gbs, "frac_hbm": pro_gbs / peaks["hbm_gbs"],
                          "bytes": pro_bytes, "traffic": pro_traffic},
             "bf16qk_attention": bf16qk,
+            "general_forms": general,
             "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": p_comp, "unit": "TFLOP/s",
                          "frac": att_tflops / p_comp, "traffic": traffic,
                          "peak_note": (f"composite FP4/BF16 peak from {peaks['source']} sustained bf16 "
@@ -411,6 +455,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-bf16qk", action="store_true", help="skip timing the BF16-QK attention")
+    ap.add_argument("--no-general", action="store_true",
+                    help="skip timing the dynamic-scale prologue and the [B,N,H,128] layout")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
