@@ -369,3 +369,136 @@ void oracle_attention_head(const float* qhat, const float* khat, const uint16_t*
         free(s);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Training-time backward (page section "NVFP4 QAD": 4-bit math on from the  */
+/* first step of distillation; the summary list: the training-time FP4       */
+/* attention matches the inference kernel).  Reading: fake quantisation with */
+/* a straight-through estimator -- the attention gradients are taken at the  */
+/* dequantised Q and K, and the quantiser passes them through unchanged, so  */
+/* only the exact transforms (rotation, key centring) are differentiated.    */
+/* ------------------------------------------------------------------------ */
+
+/* Scores of query row i against all keys (fp64), and the row's lse. */
+static double score_row(const float* q, const float* khat, int64_t N, double scale, double* s) {
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < N; ++j) {
+        const float* kk = khat + j * 128;
+        double dot = 0.0;
+        for (int c = 0; c < 128; ++c) dot += (double)q[c] * (double)kk[c];
+        s[j] = dot * scale;
+        if (s[j] > mx) mx = s[j];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < N; ++j) l += exp(s[j] - mx);
+    return mx + log(l);
+}
+
+void oracle_attention_backward_head(const float* qhat, const float* khat, const uint16_t* v, const double* dO,
+                                    int64_t N, double scale, double* dqhat, double* dkhat, double* dv) {
+    double* lse = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    double* D = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    /* pass over queries: lse_i, D_i = sum_j P_ij dP_ij, dQhat_i = scale sum_j dS_ij khat_j */
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < N; ++i) {
+            const double li = score_row(qhat + i * 128, khat, N, scale, s);
+            const double* g = dO + i * 128;
+            double Di = 0.0;
+            for (int64_t j = 0; j < N; ++j) {
+                const uint16_t* vv = v + j * 128;
+                double dp = 0.0;
+                for (int c = 0; c < 128; ++c) dp += g[c] * (double)oracle_bf16_to_f32(vv[c]);
+                s[j] = exp(s[j] - li) * dp; /* P_ij dP_ij */
+                Di += s[j];
+            }
+            lse[i] = li;
+            D[i] = Di;
+            /* second sweep for dS_ij = P_ij (dP_ij - D_i) */
+            score_row(qhat + i * 128, khat, N, scale, s);
+            double acc[128];
+            for (int c = 0; c < 128; ++c) acc[c] = 0.0;
+            for (int64_t j = 0; j < N; ++j) {
+                const uint16_t* vv = v + j * 128;
+                double dp = 0.0;
+                for (int c = 0; c < 128; ++c) dp += g[c] * (double)oracle_bf16_to_f32(vv[c]);
+                const double ds = exp(s[j] - li) * (dp - Di);
+                const float* kk = khat + j * 128;
+                for (int c = 0; c < 128; ++c) acc[c] += ds * (double)kk[c];
+            }
+            for (int c = 0; c < 128; ++c) dqhat[i * 128 + c] = scale * acc[c];
+        }
+        free(s);
+    }
+    /* pass over keys: dKhat_j = scale sum_i dS_ij qhat_i, dV_j = sum_i P_ij dO_i */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t j = 0; j < N; ++j) {
+        const float* kk = khat + j * 128;
+        const uint16_t* vv = v + j * 128;
+        double ak[128], av[128];
+        for (int c = 0; c < 128; ++c) ak[c] = av[c] = 0.0;
+        for (int64_t i = 0; i < N; ++i) {
+            const float* q = qhat + i * 128;
+            const double* g = dO + i * 128;
+            double dot = 0.0, dp = 0.0;
+            for (int c = 0; c < 128; ++c) {
+                dot += (double)q[c] * (double)kk[c];
+                dp += g[c] * (double)oracle_bf16_to_f32(vv[c]);
+            }
+            const double p = exp(dot * scale - lse[i]);
+            const double ds = p * (dp - D[i]);
+            for (int c = 0; c < 128; ++c) {
+                ak[c] += ds * (double)q[c];
+                av[c] += p * g[c];
+            }
+        }
+        for (int c = 0; c < 128; ++c) {
+            dkhat[j * 128 + c] = scale * ak[c];
+            dv[j * 128 + c] = av[c];
+        }
+    }
+    free(lse);
+    free(D);
+}
+
+/* fp64 Walsh-Hadamard transform of 128 values, the same Sylvester order as
+ * the forward (the matrix is symmetric, so it is its own transpose). */
+static void fwht128_f64(double* x) {
+    for (int h = 1; h < 128; h *= 2)
+        for (int i = 0; i < 128; ++i)
+            if ((i & h) == 0) {
+                const double a = x[i], b = x[i + h];
+                x[i] = a + b;
+                x[i + h] = a - b;
+            }
+}
+
+void oracle_ste_grads(const double* dqhat, const double* dkhat, int64_t N, uint32_t flags, double* dq, double* dk) {
+    const double c = 1.0 / sqrt(128.0);
+    double mean[128];
+    for (int ch = 0; ch < 128; ++ch) mean[ch] = 0.0;
+    if (!(flags & ORACLE_NO_SMOOTH_K) && N > 0) {
+        for (int64_t n = 0; n < N; ++n)
+            for (int ch = 0; ch < 128; ++ch) mean[ch] += dkhat[n * 128 + ch];
+        for (int ch = 0; ch < 128; ++ch) mean[ch] /= (double)N;
+    }
+    for (int64_t n = 0; n < N; ++n) {
+        double xq[128], xk[128];
+        for (int ch = 0; ch < 128; ++ch) {
+            xq[ch] = dqhat[n * 128 + ch];
+            xk[ch] = dkhat[n * 128 + ch] - mean[ch];
+        }
+        if (!(flags & ORACLE_NO_HADAMARD)) {
+            fwht128_f64(xq);
+            fwht128_f64(xk);
+            for (int ch = 0; ch < 128; ++ch) {
+                xq[ch] *= c;
+                xk[ch] *= c;
+            }
+        }
+        memcpy(dq + n * 128, xq, sizeof xq);
+        memcpy(dk + n * 128, xk, sizeof xk);
+    }
+}

@@ -113,6 +113,26 @@ void oracle_attention_head(const float* qhat, const float* khat, const uint16_t*
 /* Number of OpenMP threads the oracle uses. */
 int oracle_num_threads(void);
 
+/* Backward of oracle_attention_head for one head (fp64 throughout), the
+ * training-time gradient at the dequantised Q and K:
+ *   P = softmax(scale * qhat khat^T), O = P V, dP = dO V^T,
+ *   D_i = sum_j P_ij dP_ij, dS = P * (dP - D),
+ *   dqhat = scale * dS khat, dkhat = scale * dS^T qhat, dv = P^T dO.
+ * qhat, khat: fp32 [N,128]; v: bf16 bits [N,128]; dO: fp64 [N,128];
+ * outputs fp64 [N,128]. */
+void oracle_attention_backward_head(const float* qhat, const float* khat, const uint16_t* v_bf16,
+                                    const double* dO, int64_t N, double scale, double* dqhat,
+                                    double* dkhat, double* dv);
+
+/* Straight-through estimator of the prologue for one head: the quantiser
+ * passes gradients unchanged, the exact transforms are differentiated.
+ *   dq_n = c * H dqhat_n,  dk_n = c * H (dkhat_n - mean_n' dkhat_n'),
+ * with c = 1/sqrt(128) and H the Sylvester Hadamard matrix (symmetric); the
+ * centring is the Jacobian of the key mean (skipped with ORACLE_NO_SMOOTH_K),
+ * the rotation skipped with ORACLE_NO_HADAMARD.  fp64 in and out, [N,128]. */
+void oracle_ste_grads(const double* dqhat, const double* dkhat, int64_t N, uint32_t flags, double* dq,
+                      double* dk);
+
 #ifdef __cplusplus
 }
 #endif
