@@ -380,6 +380,37 @@ def run_ours(args, rank, world, local):
                    "bnhd_layout_step_ms": ms_t, "bnhd_layout_tflops": F / (ms_t * 1e-3) / 1e12}
         del qt, kt, vt, ot
 
+    # ---- training-time backward (straight-through), outside the timed step:
+    # dequantised Q^, K^ of this step's codes, the step's O and lse, a random dO ----
+    training = None
+    if not args.no_train:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        fa.fp4attn_quantize_qk(q, k, flags=0, out=out, workspace=ws, stream=stream)
+        fa.fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, o=o, lse=lse,
+                           workspace=ws, stream=stream)
+        qh = fa.fp4attn_dequant_bf16(out["q_codes"], out["q_scales"], stream=stream)
+        kh = fa.fp4attn_dequant_bf16(out["k_codes"], out["k_scales"], stream=stream)
+        g = torch.Generator(device=dev).manual_seed(17)
+        dout = torch.randn((B, H, N, 128), generator=g, device=dev).to(torch.bfloat16)
+        bws = torch.empty(fa.fp4attn_backward_workspace_bytes(B, H, N), dtype=torch.uint8, device=dev)
+        fa.fp4attn_backward(qh, kh, v, o, dout, lse, workspace=bws, stream=stream)
+        reps = 2
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for e in tev:
+            e[0].record(stream)
+            fa.fp4attn_backward(qh, kh, v, o, dout, lse, workspace=bws, stream=stream)
+            e[1].record(stream)
+        torch.cuda.synchronize(dev)
+        st = fa.fp4attn_read_status(bws)
+        if st != 0:
+            raise RuntimeError(f"device status after the backward: {fa.status_string(st)}")
+        ms_bw = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in tev), world, dev)
+        f_bw = 2.5 * F  # five N x N x d products against the forward's two
+        training = {"backward_ms": ms_bw, "backward_tflops": f_bw / (ms_bw * 1e-3) / 1e12,
+                    "frac_bf16_sustained": f_bw / (ms_bw * 1e-3) / 1e12 / peaks["bf16_sustained"],
+                    "launches": 5}
+        del qh, kh, dout, bws
+
     csrc = os.path.join(ROOT, "nvfp4_precision_b200", "csrc")
     traffic = ATTN_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "attention.cu")), args.workload))
     pro_traffic = PROLOGUE_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "prologue.cu")), args.workload))
@@ -430,6 +461,7 @@ def run_ours(args, rank, world, local):
                          "bytes": pro_bytes, "traffic": pro_traffic},
             "bf16qk_attention": bf16qk,
             "general_forms": general,
+            "training_backward": training,
             "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": p_comp, "unit": "TFLOP/s",
                          "frac": att_tflops / p_comp, "traffic": traffic,
                          "peak_note": (f"composite FP4/BF16 peak from {peaks['source']} sustained bf16 "
@@ -455,6 +487,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-bf16qk", action="store_true", help="skip timing the BF16-QK attention")
+    ap.add_argument("--no-train", action="store_true", help="skip timing the training-time backward")
     ap.add_argument("--no-general", action="store_true",
                     help="skip timing the dynamic-scale prologue and the [B,N,H,128] layout")
     args = ap.parse_args()

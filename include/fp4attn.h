@@ -206,6 +206,43 @@ int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, 
                                 uint8_t* k_codes_dev, uint8_t* k_scales_dev, float* k_mean_dev,
                                 int* status_dev, cudaStream_t stream);
 
+/* Training-time attention (FastVideo "Pika H3 Flex in FastVideo", section
+ * "NVFP4 QAD": the 4-bit student trains with 4-bit math on from the first
+ * step; the summary list: the training-time FP4 attention matches the
+ * inference kernel).  The forward is the inference path (fp4attn_quantize_qk,
+ * fp4attn_forward with lse) plus fp4attn_dequant_bf16 of the codes; the
+ * backward below is a straight-through estimator: attention gradients at the
+ * dequantised Q^ and K^, passed unchanged through the quantiser, then the
+ * exact transforms differentiated:
+ *   P = exp(scale Q^K^T - lse), dP = dO V^T, D = rowsum(dO * O),
+ *   dS = P * (dP - D), dV = P^T dO, dQ^ = scale dS K^, dK^ = scale dS^T Q^,
+ *   dq = c H dQ^, dk = c H (dK^ - mean_n dK^)   (c = 1/sqrt(128)).
+ * P and dS are rounded to bf16 for the BF16 tensor-core products, which
+ * accumulate in fp32; dq, dk, dv are bf16.
+ *   qhat_dev, khat_dev : [B,H,N,128] bf16 dequantised Q and K (global scale
+ *     included), e.g. from fp4attn_dequant_bf16.
+ *   v_dev, o_dev, do_dev : [B,H,N,128] bf16: V, the forward's O and dL/dO.
+ *   lse_dev : [B,H,N] fp32 from the forward.
+ *   softmax_scale : that of the forward (<= 0 selects 1/sqrt(128)).
+ *   flags : the forward's FP4ATTN_NO_SMOOTH_K / FP4ATTN_NO_HADAMARD.
+ *   dq_dev, dk_dev, dv_dev : [B,H,N,128] bf16 out: gradients of the bf16 Q,
+ *     K (the prologue's inputs) and V.
+ *   workspace_dev : fp4attn_backward_workspace_bytes(s) bytes (status word
+ *     first, so fp4attn_read_status works on it; about 512 bytes per row).
+ * All tensors contiguous.  Device errors: FP4ATTN_ERR_TIMEOUT if an internal
+ * wait ran out. */
+size_t fp4attn_backward_workspace_bytes(fp4attn_shape s);
+int fp4attn_backward(const void* qhat_dev, const void* khat_dev, const void* v_dev, const void* o_dev,
+                     const void* do_dev, const float* lse_dev, fp4attn_shape s, float softmax_scale,
+                     uint32_t flags, void* dq_dev, void* dk_dev, void* dv_dev, void* workspace_dev,
+                     size_t workspace_bytes, cudaStream_t stream);
+
+/* Decode NVFP4 rows to bf16: out = bf16(fl(fl(g * s) * e2m1)), exact when
+ * g = 1.  codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or
+ * NULL, out_dev bf16 [rows,128], rows = B*H*N of s. */
+int fp4attn_dequant_bf16(const uint8_t* codes_dev, const uint8_t* scales_dev, const float* gscale_dev,
+                         fp4attn_shape s, void* out_dev, cudaStream_t stream);
+
 /* Testing: decode NVFP4 rows back to fp32, out = fl(fl(g * s) * e2m1).
  *   codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or NULL,
  *   out_dev fp32 [rows,128], rows = B*H*N of s. */

@@ -254,6 +254,68 @@ int fp4attn_forward_bf16qk(const void* q, const void* k, const void* v, fp4attn_
                                      contiguous(s), lse, workspace, workspace_bytes, stream);
 }
 
+size_t fp4attn_backward_workspace_bytes(fp4attn_shape s) {
+    int64_t bh = heads(s);
+    if (bh < 0) bh = 0;
+    return bws_bytes(bh, s.N > 0 ? s.N : 0);
+}
+
+int fp4attn_backward(const void* qhat, const void* khat, const void* v, const void* o, const void* dout,
+                     const float* lse, fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq, void* dk,
+                     void* dv, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    int st = check_shape(s);
+    if (st != FP4ATTN_OK) return st;
+    if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD)) return FP4ATTN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < fp4attn_backward_workspace_bytes(s) || !aligned16(workspace))
+        return FP4ATTN_ERR_WORKSPACE;
+    if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f) return FP4ATTN_ERR_INVALID_ARG;
+    if (!empty(s)) {
+        const void* ptrs[] = {qhat, khat, v, o, dout, lse, dq, dk, dv};
+        for (const void* p : ptrs)
+            if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t BH = heads(s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, WS_STATUS_BYTES, stream);
+    if (e != cudaSuccess) return launch_status(e);
+    if (empty(s)) return FP4ATTN_OK;
+    BwdArgs a;
+    a.qhat = static_cast<const __nv_bfloat16*>(qhat);
+    a.khat = static_cast<const __nv_bfloat16*>(khat);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.o = static_cast<const __nv_bfloat16*>(o);
+    a.dout = static_cast<const __nv_bfloat16*>(dout);
+    a.lse = lse;
+    a.BH = (int)BH;
+    a.H = s.H;
+    a.N = s.N;
+    a.softmax_scale = softmax_scale;
+    a.flags = flags;
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.dsum = reinterpret_cast<float*>(ws + bws_dsum_offset());
+    a.colsum = reinterpret_cast<float*>(ws + bws_colsum_offset(BH, s.N));
+    a.partial = reinterpret_cast<float*>(ws + bws_partial_offset(BH, s.N));
+    a.dk_acc = reinterpret_cast<float*>(ws + bws_dk_offset(BH, s.N));
+    a.status = reinterpret_cast<int*>(ws);
+    st = launch_backward(a, stream);
+    if (st != FP4ATTN_OK) (void)cudaGetLastError();
+    return st;
+}
+
+int fp4attn_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s, void* out,
+                         cudaStream_t stream) {
+    int st = check_shape(s);
+    if (st != FP4ATTN_OK) return st;
+    if (empty(s)) return FP4ATTN_OK;
+    if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out) || ((uintptr_t)scales & 7))
+        return FP4ATTN_ERR_INVALID_ARG;
+    if (g && ((uintptr_t)g & 3)) return FP4ATTN_ERR_INVALID_ARG;
+    return launch_status(
+        launch_dequant_bf16(codes, scales, g, heads(s) * s.N, static_cast<__nv_bfloat16*>(out), stream));
+}
+
 int fp4attn_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s,
                     float* out, cudaStream_t stream) {
     int st = check_shape(s);

@@ -1,0 +1,790 @@
+// Training-time backward of the FP4 attention: fake quantisation with a
+// straight-through estimator.
+//
+// FastVideo "Pika H3 Flex in FastVideo": section "NVFP4 QAD" trains the 4-bit
+// student with 4-bit math on from the first step, and the summary list says
+// the training-time FP4 attention matches the inference kernel.  The forward
+// is the inference path itself (quantise, FP4 attention); the backward takes
+// the attention gradients at the dequantised Q^ and K^ (bf16, exact for a unit
+// global scale), passes them unchanged through the quantiser and
+// differentiates the exact transforms:
+//   dS = P * (dP - D),  P = exp(scale Q^K^T - lse),  dP = dO V^T,
+//   D_i = sum_c dO_ic O_ic,
+//   dQ^ = scale dS K^,  dK^ = scale dS^T Q^,  dV = P^T dO,
+//   dq = c H dQ^,  dk = c H (dK^ - mean_n dK^)   (c = 1/sqrt(128)).
+//
+// Three kernels, all on the fifth-generation tensor cores (BF16 operands,
+// fp32 accumulators in TMEM):
+//   bwd_q_kernel  one CTA per (head, 128 queries): D of its rows (written for
+//                 the next kernel), then per 64-key stage S = Q^K^T and
+//                 dP = dO V^T (M=128, N=64), dS in registers written as bf16
+//                 over the first 32 columns of S, dQ^ += dS K^ with dS read
+//                 from TMEM; epilogue dq = c H (scale dQ^) in registers.
+//   bwd_kv_kernel one CTA per (head, 128 keys): per 64-query stage
+//                 S^T = K^Q^T and dP^T = V dO^T, P^T and dS^T as bf16 over
+//                 them, dV += P^T dO and dK^ += dS^T Q^ with A from TMEM;
+//                 epilogue dv (bf16), scale dK^ (fp32 scratch) and each
+//                 warp's column sums of it (for the centring).
+//   colsum_kernel the head's column sums, added in a fixed order (so the
+//                 gradients are the same bits on every run).
+//   ste_k_kernel  one warp per key row: dk = c H (dK^ - colsum/N).
+// Warps: 0-3 compute (one TMEM lane = one row each), 4 the TMA producer, 5
+// the TMEM owner and MMA issuer.  TMEM (512 columns): X_b [64b, 64b+64) and
+// Y_b [128+64b, ...) for the two stage buffers b (S and dP, or S^T and dP^T),
+// accumulators at [256, 384) and [384, 512).  Every wait is bounded; a wait
+// that runs out raises FP4ATTN_ERR_TIMEOUT and the CTA winds down.
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace fp4attn {
+
+namespace {
+
+constexpr int BR = 128;     // rows of the resident tile (queries or keys)
+constexpr int BS = 64;      // rows of a streamed stage (keys or queries)
+constexpr int STAGES = 3;
+constexpr int THREADS = 192;
+constexpr int WARP_PRODUCER = 4;
+constexpr int WARP_MMA = 5;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_X = 0, TM_Y = 128, TM_ACC0 = 256, TM_ACC1 = 384;
+
+constexpr uint32_t PANEL_R = BR * 128;  // 128 rows x 64 channels bf16 (128B swizzle)
+constexpr uint32_t TILE_R = 2 * PANEL_R;
+constexpr uint32_t PANEL_S = BS * 128;  // 64 rows x 64 channels
+constexpr uint32_t TILE_S = 2 * PANEL_S;
+
+// kind::f16 with fp32 accumulation (1 << 4) and BF16 A, B (1 << 7, 1 << 10).
+//   IDESC_ST: M = 128, N = 64, both operands K-major (S, dP, S^T, dP^T).
+//   IDESC_AC: M = 128, N = 128, A from TMEM, B MN-major (1 << 16) (dQ^, dV, dK^).
+constexpr uint32_t IDESC_ST = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BS >> 3) << 17) |
+                              ((uint32_t)(BR >> 4) << 24);
+constexpr uint32_t IDESC_AC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(128 >> 3) << 17) |
+                              ((uint32_t)(BR >> 4) << 24);
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          uint64_t limit) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, status, limit);
+    return __all_sync(0xffffffffu, ok);
+}
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+    int dummy_abort = 0;
+    return mbar_wait(bar, parity, &dummy_abort, nullptr, kDrainLimitNs);
+}
+
+// K-major 128B swizzle (channels along K): 128-byte rows of 64 channels, 8-row
+// groups 1 KB apart, the second 64 channels one panel further; K step ks (16
+// channels = 32 bytes).
+__device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile) {
+    return smem_desc(smem_u32(tile), 16, 1024, LAYOUT_SW128);
+}
+__host__ __device__ constexpr uint64_t kstep(uint32_t panel, int ks) {
+    return (uint64_t)((panel * (uint32_t)(ks >> 2) + 32u * (uint32_t)(ks & 3)) >> 4);
+}
+// MN-major 128B swizzle (channels along N, rows along K): the two 64-channel
+// panels `panel` bytes apart, 8-row groups 1 KB apart; K step (16 rows) 2 KB.
+__device__ __forceinline__ uint64_t mn_desc(const uint8_t* tile, uint32_t panel) {
+    return smem_desc(smem_u32(tile), panel, 1024, LAYOUT_SW128);
+}
+constexpr uint64_t MN_KSTEP = 2048 >> 4;
+
+// In-register Walsh-Hadamard transform of 128 values (Sylvester order).
+__device__ __forceinline__ void fwht128(float* x) {
+#pragma unroll
+    for (int h = 1; h < 128; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+            if ((i & h) == 0) {
+                const float a = x[i], b = x[i + h];
+                x[i] = a + b;
+                x[i + h] = a - b;
+            }
+        }
+    }
+}
+
+struct BwdParams {
+    int N, H;
+    int n_st;          // streamed stages of BS rows
+    float scale;       // softmax scale
+    float scale_log2;  // softmax scale * log2(e)
+    const float* lse;  // [BH, N], natural log
+    float* dsum;       // [BH, N]: D, written by bwd_q_kernel, read by bwd_kv_kernel
+    const __nv_bfloat16* o;
+    const __nv_bfloat16* dout;
+    __nv_bfloat16* dq;  // [BH, N, 128]
+    __nv_bfloat16* dv;
+    float* dk_acc;      // [BH, N, 128] fp32: scale * dK^
+    float* partial;     // [BH, key tiles * 4, 128] fp32: column sums of scale * dK^ per warp
+    bool hadamard;
+    int* status;
+    uint64_t limit_ns;
+};
+
+// ------------------------------------------------------------- dQ kernel --
+
+struct __align__(1024) QSmem {
+    uint8_t q[TILE_R];               // Q^ tile, K-major
+    uint8_t dout[TILE_R];            // dO tile, K-major
+    uint8_t k[STAGES][TILE_S];       // K^ stage: K-major for S, MN-major for dQ^ += dS K^
+    uint8_t v[STAGES][TILE_S];       // V stage, K-major for dP
+    uint64_t bar_q_full;
+    uint64_t bar_kv_full[STAGES];
+    uint64_t bar_kv_empty[STAGES];
+    uint64_t bar_s_full[2];   // S_b and dP_b of a stage are in TMEM
+    uint64_t bar_p_ready[2];  // dS_b (bf16) is in TMEM
+    uint64_t bar_final;       // every MMA of the CTA has completed
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    QSmem& sm = *reinterpret_cast<QSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int q0 = blockIdx.x * BR;
+    const int T = p.n_st;
+    const int N = p.N;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&sm.bar_q_full), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&sm.bar_kv_full[s]), 1);
+            mbar_init(smem_u32(&sm.bar_kv_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&sm.bar_s_full[b]), 1);
+            mbar_init(smem_u32(&sm.bar_p_ready[b]), 128);
+        }
+        mbar_init(smem_u32(&sm.bar_final), 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(smem_u32(&sm.tmem_base), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* abort_flag = &sm.abort_flag;
+    const uint64_t limit = p.limit_ns;
+    const int hb = bh / p.H, hh = bh - hb * p.H;
+
+    if (warp == WARP_PRODUCER) {
+        // Q^ and dO once, then K^ and V of BS keys per stage.  Rows past N are
+        // filled with zeros by the copy.
+        const uint32_t qf = smem_u32(&sm.bar_q_full);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(qf, 2 * TILE_R);
+            tma_load_4d(smem_u32(sm.q), &tm_q, 0, q0, hh, hb, qf);
+            tma_load_4d(smem_u32(sm.q) + PANEL_R, &tm_q, 64, q0, hh, hb, qf);
+            tma_load_4d(smem_u32(sm.dout), &tm_do, 0, q0, hh, hb, qf);
+            tma_load_4d(smem_u32(sm.dout) + PANEL_R, &tm_do, 64, q0, hh, hb, qf);
+        }
+        int issued = 0;
+        for (int j = 0; j < T; ++j) {
+            const int st = j % STAGES;
+            if (j >= STAGES &&
+                !warp_wait(smem_u32(&sm.bar_kv_empty[st]), ((j / STAGES) - 1) & 1, abort_flag, p.status, limit))
+                break;
+            if (lane == 0) {
+                const uint32_t full = smem_u32(&sm.bar_kv_full[st]);
+                const int k0 = j * BS;
+                mbar_arrive_expect_tx(full, 2 * TILE_S);
+                tma_load_4d(smem_u32(sm.k[st]), &tm_k, 0, k0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.k[st]) + PANEL_S, &tm_k, 64, k0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.v[st]), &tm_v, 0, k0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.v[st]) + PANEL_S, &tm_v, 64, k0, hh, hb, full);
+            }
+            __syncwarp();
+            issued = j + 1;
+        }
+        if (lane == 0 && *abort_flag) {
+            drain_wait(qf, 0);
+            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+                drain_wait(smem_u32(&sm.bar_kv_full[i % STAGES]), (i / STAGES) & 1);
+        }
+    } else if (warp == WARP_MMA) {
+        const bool leader = elect_one_sync();
+        const uint64_t qd = kmajor_desc(sm.q);
+        const uint64_t dod = kmajor_desc(sm.dout);
+        const uint64_t kd0 = kmajor_desc(sm.k[0]);   // stage st: + st * TILE_S / 16
+        const uint64_t vd0 = kmajor_desc(sm.v[0]);
+        const uint64_t kmn0 = mn_desc(sm.k[0], PANEL_S);
+        constexpr uint64_t TD = TILE_S >> 4;
+        auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, p.status, limit));
+        };
+        auto scores = [&](int b, int st) {  // S_b = Q^ K^T, dP_b = dO V^T
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+                mma_bf16_ss(tmem + TM_X + BS * b, qd + kstep(PANEL_R, ks), kd0 + TD * st + kstep(PANEL_S, ks),
+                            IDESC_ST, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+                mma_bf16_ss(tmem + TM_Y + BS * b, dod + kstep(PANEL_R, ks), vd0 + TD * st + kstep(PANEL_S, ks),
+                            IDESC_ST, ks > 0 ? 1u : 0u);
+            tc_commit(smem_u32(&sm.bar_s_full[b]));
+        };
+        auto accumulate = [&](int b, int st, bool acc) {  // dQ^ += dS_b K^ (dS from TMEM)
+#pragma unroll
+            for (int ks = 0; ks < BS / 16; ++ks)
+                mma_bf16_ts(tmem + TM_ACC0, tmem + TM_X + BS * b + 8u * ks, kmn0 + TD * st + MN_KSTEP * ks,
+                            IDESC_AC, (acc || ks > 0) ? 1u : 0u);
+            tc_commit(smem_u32(&sm.bar_kv_empty[st]));
+        };
+        bool ok = wait(smem_u32(&sm.bar_q_full), 0);
+        for (int j = 0; ok && j < T; ++j) {
+            const int st = j % STAGES;
+            if (!wait(smem_u32(&sm.bar_kv_full[st]), (j / STAGES) & 1)) {
+                ok = false;
+                break;
+            }
+            if (leader) {
+                tc_fence_after();
+                scores(j & 1, st);
+            }
+            __syncwarp();
+            if (j > 0) {
+                if (!wait(smem_u32(&sm.bar_p_ready[(j - 1) & 1]), ((j - 1) >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (leader) {
+                    tc_fence_after();
+                    accumulate((j - 1) & 1, (j - 1) % STAGES, j > 1);
+                }
+                __syncwarp();
+            }
+        }
+        if (ok && T > 0 && wait(smem_u32(&sm.bar_p_ready[(T - 1) & 1]), ((T - 1) >> 1) & 1)) {
+            if (leader) {
+                tc_fence_after();
+                accumulate((T - 1) & 1, (T - 1) % STAGES, T > 1);
+            }
+            __syncwarp();
+        }
+        // the final commit tells the compute warps that dQ^ is complete, and
+        // is what this warp waits on before TMEM is freed
+        if (leader) {
+            tc_commit(smem_u32(&sm.bar_final));
+            drain_wait(smem_u32(&sm.bar_final), 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ compute warps --
+        const int row = 32 * warp + lane;
+        const int n = q0 + row;
+        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const size_t grow = (size_t)bh * N + n;
+        // D = sum_c dO_c O_c of this row, and the row's lse in the log2 domain;
+        // rows past N get p = 0 (lse = +inf) and D = 0
+        float Dr = 0.0f, lse2 = INFINITY;
+        if (n < N) {
+            const uint4* po = reinterpret_cast<const uint4*>(p.o + grow * 128);
+            const uint4* pd = reinterpret_cast<const uint4*>(p.dout + grow * 128);
+            float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll 4
+            for (int c = 0; c < 16; ++c) {
+                const uint4 a = po[c], g = pd[c];
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc = __ffma2_rn(make_float2(bf16lo(aw[e]), bf16hi(aw[e])),
+                                     make_float2(bf16lo(gw[e]), bf16hi(gw[e])), acc);
+            }
+            Dr = acc.x + acc.y;
+            p.dsum[grow] = Dr;
+            lse2 = p.lse[grow] * kLog2e;
+        }
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int j = 0; j < T; ++j) {
+            const int b = j & 1;
+            if (!warp_wait(smem_u32(&sm.bar_s_full[b]), (j >> 1) & 1, abort_flag, p.status, limit)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sr[BS], dr[BS];
+            tmem_ld32(tmem + lane_base + TM_X + BS * b, &sr[0]);
+            tmem_ld32(tmem + lane_base + TM_X + BS * b + 32, &sr[32]);
+            tmem_ld32(tmem + lane_base + TM_Y + BS * b, &dr[0]);
+            tmem_ld32(tmem + lane_base + TM_Y + BS * b + 32, &dr[32]);
+            tmem_wait_ld();
+            const int nvalid = N - j * BS;  // keys of this stage that exist
+            uint32_t pk[BS / 2];
+#pragma unroll
+            for (int k = 0; k < BS / 2; ++k) {
+                float ds[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int kk = 2 * k + e;
+                    const float pr = ex2_approx(fmaf(__uint_as_float(sr[kk]), c, -lse2));
+                    ds[e] = (kk < nvalid) ? pr * (__uint_as_float(dr[kk]) - Dr) : 0.0f;
+                }
+                pk[k] = pack_bf16x2(ds[0], ds[1]);
+            }
+            tmem_st32(tmem + lane_base + TM_X + BS * b, pk);  // dS over the first 32 columns of S_b
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.bar_p_ready[b]));
+        }
+        if (ok && T > 0 && warp_wait(smem_u32(&sm.bar_final), 0, abort_flag, p.status, limit)) {
+            tc_fence_after();
+            float x[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + TM_ACC0 + 32u * q, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[32 * q + e] = __uint_as_float(r[e]) * p.scale;
+            }
+            if (p.hadamard) {
+                fwht128(x);
+                const float h = __uint_as_float(0x3DB504F3u);  // fp32(1/sqrt(128))
+#pragma unroll
+                for (int e = 0; e < 128; ++e) x[e] *= h;
+            }
+            if (n < N) {
+                uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * 128);
+#pragma unroll
+                for (int v = 0; v < 16; ++v)
+                    dst[v] = make_uint4(pack_bf16x2(x[8 * v], x[8 * v + 1]), pack_bf16x2(x[8 * v + 2], x[8 * v + 3]),
+                                        pack_bf16x2(x[8 * v + 4], x[8 * v + 5]),
+                                        pack_bf16x2(x[8 * v + 6], x[8 * v + 7]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------- dK, dV kernel --
+
+struct __align__(1024) KVSmem {
+    uint8_t k[TILE_R];                // K^ tile, K-major (A of S^T)
+    uint8_t v[TILE_R];                // V tile, K-major (A of dP^T)
+    uint8_t q[STAGES][TILE_S];        // Q^ stage: K-major for S^T, MN-major for dK^ += dS^T Q^
+    uint8_t dout[STAGES][TILE_S];     // dO stage: K-major for dP^T, MN-major for dV += P^T dO
+    float lse2[STAGES][BS];           // lse * log2(e) of the stage's queries (+inf past N)
+    float dsum[STAGES][BS];           // D of the stage's queries (0 past N)
+    uint64_t bar_kv_full;
+    uint64_t bar_q_full[STAGES];
+    uint64_t bar_q_empty[STAGES];
+    uint64_t bar_s_full[2];
+    uint64_t bar_p_ready[2];
+    uint64_t bar_final;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// Sum of each of 128 columns over the 32 lanes of a warp: after five rounds of
+// exchanging half of the remaining partial sums, lane l holds the sums of
+// columns 4l .. 4l+3 in a[0..3].
+template <int R>
+__device__ __forceinline__ void column_sum_round(float* a, int lane) {
+    constexpr int half = 64 >> R;  // partial sums exchanged this round
+    const bool upper = (lane >> (4 - R)) & 1;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+        const float send = upper ? a[i] : a[i + half];
+        const float keep = upper ? a[i + half] : a[i];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16 >> R);
+    }
+}
+__device__ __forceinline__ void warp_column_sums(float* a, int lane) {
+    column_sum_round<0>(a, lane);
+    column_sum_round<1>(a, lane);
+    column_sum_round<2>(a, lane);
+    column_sum_round<3>(a, lane);
+    column_sum_round<4>(a, lane);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    KVSmem& sm = *reinterpret_cast<KVSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int k0 = blockIdx.x * BR;
+    const int T = p.n_st;
+    const int N = p.N;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&sm.bar_kv_full), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&sm.bar_q_full[s]), 32);  // every producer lane (its lse / D stores)
+            mbar_init(smem_u32(&sm.bar_q_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&sm.bar_s_full[b]), 1);
+            mbar_init(smem_u32(&sm.bar_p_ready[b]), 128);
+        }
+        mbar_init(smem_u32(&sm.bar_final), 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(smem_u32(&sm.tmem_base), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int* abort_flag = &sm.abort_flag;
+    const uint64_t limit = p.limit_ns;
+    const int hb = bh / p.H, hh = bh - hb * p.H;
+
+    if (warp == WARP_PRODUCER) {
+        const uint32_t kvf = smem_u32(&sm.bar_kv_full);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kvf, 2 * TILE_R);
+            tma_load_4d(smem_u32(sm.k), &tm_k, 0, k0, hh, hb, kvf);
+            tma_load_4d(smem_u32(sm.k) + PANEL_R, &tm_k, 64, k0, hh, hb, kvf);
+            tma_load_4d(smem_u32(sm.v), &tm_v, 0, k0, hh, hb, kvf);
+            tma_load_4d(smem_u32(sm.v) + PANEL_R, &tm_v, 64, k0, hh, hb, kvf);
+        }
+        const float* lse_head = p.lse + (size_t)bh * N;
+        const float* d_head = p.dsum + (size_t)bh * N;
+        int issued = 0;
+        for (int i = 0; i < T; ++i) {
+            const int st = i % STAGES;
+            if (i >= STAGES &&
+                !warp_wait(smem_u32(&sm.bar_q_empty[st]), ((i / STAGES) - 1) & 1, abort_flag, p.status, limit))
+                break;
+#pragma unroll
+            for (int e = lane; e < BS; e += 32) {
+                const int qi = i * BS + e;
+                sm.lse2[st][e] = (qi < N) ? lse_head[qi] * kLog2e : INFINITY;
+                sm.dsum[st][e] = (qi < N) ? d_head[qi] : 0.0f;
+            }
+            const uint32_t full = smem_u32(&sm.bar_q_full[st]);
+            if (lane == 0) {
+                const int r0 = i * BS;
+                mbar_arrive_expect_tx(full, 2 * TILE_S);
+                tma_load_4d(smem_u32(sm.q[st]), &tm_q, 0, r0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.q[st]) + PANEL_S, &tm_q, 64, r0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.dout[st]), &tm_do, 0, r0, hh, hb, full);
+                tma_load_4d(smem_u32(sm.dout[st]) + PANEL_S, &tm_do, 64, r0, hh, hb, full);
+            } else {
+                mbar_arrive(full);
+            }
+            __syncwarp();
+            issued = i + 1;
+        }
+        if (lane == 0 && *abort_flag) {
+            drain_wait(kvf, 0);
+            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+                drain_wait(smem_u32(&sm.bar_q_full[i % STAGES]), (i / STAGES) & 1);
+        }
+    } else if (warp == WARP_MMA) {
+        const bool leader = elect_one_sync();
+        const uint64_t kd = kmajor_desc(sm.k);
+        const uint64_t vd = kmajor_desc(sm.v);
+        const uint64_t qd0 = kmajor_desc(sm.q[0]);  // stage st: + st * TILE_S / 16
+        const uint64_t dod0 = kmajor_desc(sm.dout[0]);
+        const uint64_t qmn0 = mn_desc(sm.q[0], PANEL_S);
+        const uint64_t domn0 = mn_desc(sm.dout[0], PANEL_S);
+        constexpr uint64_t TD = TILE_S >> 4;
+        auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, p.status, limit));
+        };
+        auto scores = [&](int b, int st) {  // S^T_b = K^ Q^T, dP^T_b = V dO^T
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+                mma_bf16_ss(tmem + TM_X + BS * b, kd + kstep(PANEL_R, ks), qd0 + TD * st + kstep(PANEL_S, ks),
+                            IDESC_ST, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+                mma_bf16_ss(tmem + TM_Y + BS * b, vd + kstep(PANEL_R, ks), dod0 + TD * st + kstep(PANEL_S, ks),
+                            IDESC_ST, ks > 0 ? 1u : 0u);
+            tc_commit(smem_u32(&sm.bar_s_full[b]));
+        };
+        auto accumulate = [&](int b, int st, bool acc) {  // dV += P^T dO, dK^ += dS^T Q^
+#pragma unroll
+            for (int ks = 0; ks < BS / 16; ++ks)
+                mma_bf16_ts(tmem + TM_ACC0, tmem + TM_X + BS * b + 8u * ks, domn0 + TD * st + MN_KSTEP * ks,
+                            IDESC_AC, (acc || ks > 0) ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < BS / 16; ++ks)
+                mma_bf16_ts(tmem + TM_ACC1, tmem + TM_Y + BS * b + 8u * ks, qmn0 + TD * st + MN_KSTEP * ks,
+                            IDESC_AC, (acc || ks > 0) ? 1u : 0u);
+            tc_commit(smem_u32(&sm.bar_q_empty[st]));
+        };
+        bool ok = wait(smem_u32(&sm.bar_kv_full), 0);
+        for (int i = 0; ok && i < T; ++i) {
+            const int st = i % STAGES;
+            if (!wait(smem_u32(&sm.bar_q_full[st]), (i / STAGES) & 1)) {
+                ok = false;
+                break;
+            }
+            if (leader) {
+                tc_fence_after();
+                scores(i & 1, st);
+            }
+            __syncwarp();
+            if (i > 0) {
+                if (!wait(smem_u32(&sm.bar_p_ready[(i - 1) & 1]), ((i - 1) >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if (leader) {
+                    tc_fence_after();
+                    accumulate((i - 1) & 1, (i - 1) % STAGES, i > 1);
+                }
+                __syncwarp();
+            }
+        }
+        if (ok && T > 0 && wait(smem_u32(&sm.bar_p_ready[(T - 1) & 1]), ((T - 1) >> 1) & 1)) {
+            if (leader) {
+                tc_fence_after();
+                accumulate((T - 1) & 1, (T - 1) % STAGES, T > 1);
+            }
+            __syncwarp();
+        }
+        if (leader) {
+            tc_commit(smem_u32(&sm.bar_final));
+            drain_wait(smem_u32(&sm.bar_final), 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ compute warps --
+        const int row = 32 * warp + lane;  // key row of the tile
+        const int kn = k0 + row;
+        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int i = 0; i < T; ++i) {
+            const int b = i & 1;
+            const int st = i % STAGES;
+            // the stage's lse / D (written by the producer lanes) and S^T, dP^T
+            if (!warp_wait(smem_u32(&sm.bar_q_full[st]), (i / STAGES) & 1, abort_flag, p.status, limit) ||
+                !warp_wait(smem_u32(&sm.bar_s_full[b]), (i >> 1) & 1, abort_flag, p.status, limit)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sr[BS], dr[BS];
+            tmem_ld32(tmem + lane_base + TM_X + BS * b, &sr[0]);
+            tmem_ld32(tmem + lane_base + TM_X + BS * b + 32, &sr[32]);
+            tmem_ld32(tmem + lane_base + TM_Y + BS * b, &dr[0]);
+            tmem_ld32(tmem + lane_base + TM_Y + BS * b + 32, &dr[32]);
+            tmem_wait_ld();
+            const float4* l4 = reinterpret_cast<const float4*>(sm.lse2[st]);
+            const float4* d4 = reinterpret_cast<const float4*>(sm.dsum[st]);
+            uint32_t pk[BS / 2], dk[BS / 2];
+#pragma unroll
+            for (int g = 0; g < BS / 4; ++g) {
+                const float4 lv = l4[g], dv = d4[g];
+                const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
+                float pr[4], ds[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int kk = 4 * g + e;
+                    pr[e] = ex2_approx(fmaf(__uint_as_float(sr[kk]), c, -la[e]));
+                    ds[e] = pr[e] * (__uint_as_float(dr[kk]) - da[e]);
+                }
+                pk[2 * g] = pack_bf16x2(pr[0], pr[1]);
+                pk[2 * g + 1] = pack_bf16x2(pr[2], pr[3]);
+                dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
+                dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
+            }
+            tmem_st32(tmem + lane_base + TM_X + BS * b, pk);  // P^T over S^T_b
+            tmem_st32(tmem + lane_base + TM_Y + BS * b, dk);  // dS^T over dP^T_b
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.bar_p_ready[b]));
+        }
+        if (ok && T > 0 && warp_wait(smem_u32(&sm.bar_final), 0, abort_flag, p.status, limit)) {
+            tc_fence_after();
+            const size_t grow = (size_t)bh * N + kn;
+            const bool valid = kn < N;
+            // dV (bf16)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + TM_ACC0 + 32u * q, r);
+                tmem_wait_ld();
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.dv + grow * 128 + 32 * q);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(
+                            pack_bf16x2(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+                }
+            }
+            // scale * dK^ (fp32) and its column sums over the valid keys
+            float x[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + TM_ACC1 + 32u * q, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[32 * q + e] = valid ? __uint_as_float(r[e]) * p.scale : 0.0f;
+            }
+            if (valid) {
+                float4* dst = reinterpret_cast<float4*>(p.dk_acc + grow * 128);
+#pragma unroll
+                for (int v = 0; v < 32; ++v) dst[v] = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+            }
+            warp_column_sums(x, lane);
+            float4* part = reinterpret_cast<float4*>(
+                p.partial + (((size_t)bh * gridDim.x + blockIdx.x) * 4 + warp) * 128);
+            part[lane] = make_float4(x[0], x[1], x[2], x[3]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------- key straight-through --
+
+// Column sums of scale * dK^ of each head: thread c of block bh adds the
+// per-warp partial sums of column c in order.
+__global__ void __launch_bounds__(128) colsum_kernel(const float* __restrict__ partial, int parts,
+                                                     float* __restrict__ colsum) {
+    const float* src = partial + (size_t)blockIdx.x * parts * 128 + threadIdx.x;
+    float acc = 0.0f;
+    for (int i = 0; i < parts; ++i) acc += src[(size_t)i * 128];
+    colsum[(size_t)blockIdx.x * 128 + threadIdx.x] = acc;
+}
+
+// One warp per key row: dk = c H (scale dK^ - colsum / N) as bf16.  Lane l
+// holds channels 4l .. 4l+3; butterfly strides 1 and 2 stay in the lane,
+// strides 4 .. 64 pair lanes l and l ^ (stride / 4).
+__global__ void __launch_bounds__(256) ste_k_kernel(const float* __restrict__ dk_acc, const float* __restrict__ colsum,
+                                                    int N, int64_t rows, bool smooth, bool hadamard,
+                                                    __nv_bfloat16* __restrict__ dk) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const float nf = (float)N;
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nw) {
+        const float4 v = reinterpret_cast<const float4*>(dk_acc + r * 128)[lane];
+        float x[4] = {v.x, v.y, v.z, v.w};
+        if (smooth) {
+            const float4 m = reinterpret_cast<const float4*>(colsum + (r / N) * 128)[lane];
+            x[0] -= __fdiv_rn(m.x, nf);
+            x[1] -= __fdiv_rn(m.y, nf);
+            x[2] -= __fdiv_rn(m.z, nf);
+            x[3] -= __fdiv_rn(m.w, nf);
+        }
+        if (hadamard) {
+            float a = x[0] + x[1], b = x[0] - x[1], cc = x[2] + x[3], d = x[2] - x[3];
+            x[0] = a + cc;
+            x[2] = a - cc;
+            x[1] = b + d;
+            x[3] = b - d;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const bool upper = lane & m;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+                    x[e] = upper ? (o - x[e]) : (x[e] + o);
+                }
+            }
+            const float h = __uint_as_float(0x3DB504F3u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] *= h;
+        }
+        reinterpret_cast<uint2*>(dk + r * 128)[lane] = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+    }
+}
+
+// [B][H][N][128 bf16], contiguous: 128B-swizzled boxes of 64 channels x
+// box_rows rows of one head (x is 0 or 64: 16-byte aligned).
+bool make_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, uint32_t box_rows) {
+    const Strides st = contiguous_strides(H, N);
+    const uint64_t dims[4] = {128, (uint64_t)N, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
+    const uint32_t box[4] = {64, box_rows, 1, 1};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(base), dims,
+                             strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+int launch_backward(const BwdArgs& a, cudaStream_t stream) {
+    if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
+    const int B = a.BH / a.H;
+    CUtensorMap q_r, do_r, k_s, v_s, k_r, v_r, q_s, do_s;
+    if (!make_map(&q_r, a.qhat, B, a.H, a.N, BR) || !make_map(&do_r, a.dout, B, a.H, a.N, BR) ||
+        !make_map(&k_s, a.khat, B, a.H, a.N, BS) || !make_map(&v_s, a.v, B, a.H, a.N, BS) ||
+        !make_map(&k_r, a.khat, B, a.H, a.N, BR) || !make_map(&v_r, a.v, B, a.H, a.N, BR) ||
+        !make_map(&q_s, a.qhat, B, a.H, a.N, BS) || !make_map(&do_s, a.dout, B, a.H, a.N, BS))
+        return FP4ATTN_ERR_CUDA;
+    static_assert(sizeof(QSmem) + 1024 <= 227 * 1024, "shared memory budget");
+    static_assert(sizeof(KVSmem) + 1024 <= 227 * 1024, "shared memory budget");
+    const size_t smem_q = sizeof(QSmem) + 1024, smem_kv = sizeof(KVSmem) + 1024;
+    if (cudaFuncSetAttribute(bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv) !=
+            cudaSuccess)
+        return FP4ATTN_ERR_CUDA;
+    BwdParams p;
+    p.N = a.N;
+    p.H = a.H;
+    p.n_st = (a.N + BS - 1) / BS;
+    p.scale = a.softmax_scale > 0.0f ? a.softmax_scale : 0.08838834764831845f;
+    p.scale_log2 = p.scale * kLog2e;
+    p.lse = a.lse;
+    p.dsum = a.dsum;
+    p.o = a.o;
+    p.dout = a.dout;
+    p.dq = a.dq;
+    p.dv = a.dv;
+    p.dk_acc = a.dk_acc;
+    p.partial = a.partial;
+    p.hadamard = !(a.flags & FP4ATTN_NO_HADAMARD);
+    p.status = a.status;
+    p.limit_ns = kWaitLimitNs;
+    const dim3 grid((a.N + BR - 1) / BR, a.BH);
+    bwd_q_kernel<<<grid, THREADS, smem_q, stream>>>(q_r, do_r, k_s, v_s, p);
+    if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
+    bwd_kv_kernel<<<grid, THREADS, smem_kv, stream>>>(k_r, v_r, q_s, do_s, p);
+    if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
+    if (!(a.flags & FP4ATTN_NO_SMOOTH_K)) {
+        colsum_kernel<<<a.BH, 128, 0, stream>>>(a.partial, 4 * (int)grid.x, a.colsum);
+        if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
+    }
+    const int64_t rows = (int64_t)a.BH * a.N;
+    const int64_t want = (rows + 7) / 8;  // 8 warps per block, one row each
+    const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+    ste_k_kernel<<<blocks, 256, 0, stream>>>(a.dk_acc, a.colsum, a.N, rows, !(a.flags & FP4ATTN_NO_SMOOTH_K),
+                                             p.hadamard, a.dk);
+    return cudaGetLastError() == cudaSuccess ? FP4ATTN_OK : FP4ATTN_ERR_CUDA;
+}
+
+}  // namespace fp4attn

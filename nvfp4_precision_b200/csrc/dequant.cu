@@ -26,6 +26,27 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t*
     for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
+// The same values rounded to bf16 (exact for a unit global scale: a 4-bit
+// times a 2-bit significand): the dequantised Q and K of the training backward.
+__global__ void dequant_bf16_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                    const float* g_ptr, int64_t nblocks, __nv_bfloat16* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nblocks) return;
+    const float g = g_ptr ? *g_ptr : 1.0f;
+    const float gs = __fmul_rn(g, ue4m3_value(scales[i]));
+    const uint2 c = *reinterpret_cast<const uint2*>(codes + i * 8);
+    uint32_t w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const uint32_t word = (e < 4) ? c.x : c.y;
+        const uint32_t lo = (word >> (8 * (e & 3))) & 0xF, hi = (word >> (8 * (e & 3) + 4)) & 0xF;
+        w[e] = pack_bf16x2(__fmul_rn(gs, e2m1_value(lo)), __fmul_rn(gs, e2m1_value(hi)));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + i * 16);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 __global__ void encode_kernel(const float* __restrict__ x, int64_t n, uint8_t* e2m1, uint8_t* e4m3) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -44,6 +65,16 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const fl
     const int threads = 256;
     dequant_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, stream>>>(
         codes, scales, g, nblocks, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+                                __nv_bfloat16* out, cudaStream_t stream) {
+    const int64_t nblocks = rows * 8;
+    if (nblocks == 0) return cudaSuccess;
+    const int threads = 256;
+    dequant_bf16_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, stream>>>(codes, scales, g,
+                                                                                               nblocks, out);
     return cudaGetLastError();
 }
 

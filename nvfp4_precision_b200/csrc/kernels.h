@@ -99,7 +99,44 @@ struct FwdBf16Args {
     int* status;
 };
 
+// Backward workspace: [0,256) status word and spare; then D [BH*N] fp32,
+// column sums [BH*128] fp32, per-warp column sums [BH*ceil(N/128)*4*128] fp32,
+// scale * dK^ [BH*N*128] fp32 (each 256-aligned).
+inline size_t bws_align(size_t b) { return (b + 255) / 256 * 256; }
+inline size_t bws_dsum_offset() { return WS_STATUS_BYTES; }
+inline size_t bws_colsum_offset(int64_t BH, int64_t N) { return bws_dsum_offset() + bws_align((size_t)(BH * N) * 4); }
+inline size_t bws_partial_offset(int64_t BH, int64_t N) {
+    return bws_colsum_offset(BH, N) + bws_align((size_t)BH * D * 4);
+}
+inline size_t bws_dk_offset(int64_t BH, int64_t N) {
+    return bws_partial_offset(BH, N) + bws_align((size_t)BH * ((N + 127) / 128) * 4 * D * 4);
+}
+inline size_t bws_bytes(int64_t BH, int64_t N) { return bws_dk_offset(BH, N) + bws_align((size_t)(BH * N) * D * 4); }
+
+struct BwdArgs {
+    const __nv_bfloat16* qhat;  // dequantised Q and K, [B,H,N,128] contiguous
+    const __nv_bfloat16* khat;
+    const __nv_bfloat16* v;
+    const __nv_bfloat16* o;
+    const __nv_bfloat16* dout;
+    const float* lse;  // [B,H,N]
+    int BH, H, N;
+    float softmax_scale;
+    uint32_t flags;  // FP4ATTN_NO_SMOOTH_K / FP4ATTN_NO_HADAMARD of the forward
+    __nv_bfloat16* dq;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* dsum;
+    float* colsum;
+    float* partial;
+    float* dk_acc;
+    int* status;
+};
+
 // Returns 0 on success, else an fp4attn_status code.
+int launch_backward(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+                                __nv_bfloat16* out, cudaStream_t stream);
 int launch_forward(const FwdArgs& a, cudaStream_t stream);
 int launch_forward_bf16qk(const FwdBf16Args& a, cudaStream_t stream);
 int launch_probe_qk(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,

@@ -30,7 +30,7 @@ DYNAMIC_GSCALE = 4
 EXPORTS = (
     "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_quantize_qk_ex", "fp4attn_quantize_qk_noalloc",
     "fp4attn_forward", "fp4attn_forward_ex", "fp4attn_forward_bf16qk", "fp4attn_forward_bf16qk_ex",
-    "fp4attn_dequant",
+    "fp4attn_dequant", "fp4attn_dequant_bf16", "fp4attn_backward", "fp4attn_backward_workspace_bytes",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
 )
@@ -76,6 +76,12 @@ def _load():
     L.fp4attn_forward.argtypes = [P, P, P, P, P, P, P, Shape, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
     L.fp4attn_forward_bf16qk.restype = ctypes.c_int
     L.fp4attn_forward_bf16qk.argtypes = [P, P, P, Shape, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_dequant_bf16.restype = ctypes.c_int
+    L.fp4attn_dequant_bf16.argtypes = [P, P, P, Shape, P, P]
+    L.fp4attn_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.fp4attn_backward_workspace_bytes.argtypes = [Shape]
+    L.fp4attn_backward.restype = ctypes.c_int
+    L.fp4attn_backward.argtypes = [P, P, P, P, P, P, Shape, ctypes.c_float, U32, P, P, P, P, ctypes.c_size_t, P]
     L.fp4attn_dequant.restype = ctypes.c_int
     L.fp4attn_dequant.argtypes = [P, P, P, Shape, P, P]
     L.fp4attn_read_status.restype = ctypes.c_int
@@ -260,6 +266,79 @@ def fp4attn_dequant(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[
                              _stream(stream))
     _check(rc, "fp4attn_dequant")
     return out
+
+
+def fp4attn_dequant_bf16(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """NVFP4 [B,H,N,64] codes + [B,H,N,8] scales -> bf16 [B,H,N,128] values."""
+    B, H, N, _ = codes.shape
+    out = torch.empty((B, H, N, 128), dtype=torch.bfloat16, device=codes.device)
+    rc = lib.fp4attn_dequant_bf16(_ptr(codes), _ptr(scales), _ptr(gscale), Shape(B, H, N, 128), _ptr(out),
+                                  _stream(stream))
+    _check(rc, "fp4attn_dequant_bf16")
+    return out
+
+
+def fp4attn_backward_workspace_bytes(B: int, H: int, N: int, D: int = 128) -> int:
+    return int(lib.fp4attn_backward_workspace_bytes(Shape(B, H, N, D)))
+
+
+def fp4attn_backward(qhat, khat, v, o, dout, lse, softmax_scale: float = 0.0, flags: int = 0,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """Straight-through backward of the FP4 attention (see include/fp4attn.h):
+    bf16 [B,H,N,128] dequantised Q^, K^, V, the forward's O, dL/dO, fp32 lse
+    [B,H,N].  Returns (dq, dk, dv, workspace), bf16 gradients of the bf16 Q,
+    K, V inputs of the forward."""
+    for t in (qhat, khat, v, o, dout):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == v.shape
+    assert lse.dtype == torch.float32 and lse.is_contiguous()
+    B, H, N, D = v.shape
+    if workspace is None:
+        workspace = torch.empty(fp4attn_backward_workspace_bytes(B, H, N), dtype=torch.uint8, device=v.device)
+    dq, dk, dv = (torch.empty((B, H, N, D), dtype=torch.bfloat16, device=v.device) for _ in range(3))
+    rc = lib.fp4attn_backward(_ptr(qhat), _ptr(khat), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), Shape(B, H, N, D),
+                              float(softmax_scale), int(flags), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                              workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_backward")
+    return dq, dk, dv, workspace
+
+
+class FP4AttentionSTE(torch.autograd.Function):
+    """Training-time FP4 attention: the inference path forward (quantise,
+    FP4 attention), straight-through backward (fp4attn_backward).  The device
+    status words of both halves are checked on the host."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, softmax_scale=0.0, flags=0):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        out = fp4attn_quantize_qk(q, k, flags=flags, k_mean=False)
+        o, lse = fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v,
+                                 softmax_scale=softmax_scale, want_lse=True, workspace=out["workspace"])
+        qhat = fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])
+        khat = fp4attn_dequant_bf16(out["k_codes"], out["k_scales"])
+        st = fp4attn_read_status(out["workspace"])
+        if st != OK:
+            raise Fp4AttnError(st, "FP4AttentionSTE.forward (device)")
+        ctx.save_for_backward(qhat, khat, v, o, lse)
+        ctx.softmax_scale, ctx.flags = softmax_scale, flags
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        qhat, khat, v, o, lse = ctx.saved_tensors
+        dq, dk, dv, ws = fp4attn_backward(qhat, khat, v, o, do.contiguous().to(torch.bfloat16), lse,
+                                          ctx.softmax_scale, ctx.flags)
+        st = fp4attn_read_status(ws)
+        if st != OK:
+            raise Fp4AttnError(st, "FP4AttentionSTE.backward (device)")
+        return dq, dk, dv, None, None
+
+
+def fp4_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float = 0.0,
+                  flags: int = 0) -> torch.Tensor:
+    """Differentiable FP4 attention of bf16 [B,H,N,128] Q, K, V (fake
+    quantisation with a straight-through backward)."""
+    return FP4AttentionSTE.apply(q, k, v, softmax_scale, flags)
 
 
 def fp4attn_read_status(workspace: torch.Tensor, stream=None) -> int:

@@ -61,7 +61,7 @@ def lib():
         L.oracle_dynamic_gscale.argtypes = [P, P, i64, i64, i64, ctypes.c_uint32, P, P]
         L.oracle_dequant.argtypes = [P, P, ctypes.c_float, i64, P]
         L.oracle_attention_head.argtypes = [P, P, P, i64, ctypes.c_double, P, i64, P, P]
-        L.oracle_attention_backward_head.argtypes = [P, P, P, P, i64, ctypes.c_double, P, P, P]
+        L.oracle_attention_backward_head.argtypes = [P, P, P, P, P, i64, ctypes.c_double, P, P, P]
         L.oracle_ste_grads.argtypes = [P, P, i64, ctypes.c_uint32, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
@@ -250,10 +250,13 @@ def attention(q_codes, q_scales, k_codes, k_scales, v_bits, gq=1.0, gk=1.0, scal
 
 # -- training-time backward (fake quantisation, straight-through estimator) ------
 
-def attention_backward_head(qhat: np.ndarray, khat: np.ndarray, v_bits: np.ndarray, dO: np.ndarray, scale=None):
+def attention_backward_head(qhat: np.ndarray, khat: np.ndarray, v_bits: np.ndarray, dO: np.ndarray, scale=None,
+                            O=None):
     """fp64 gradients of one head's attention at the dequantised Q and K.
     qhat, khat: float32 [N,128]; v_bits: bf16 bits [N,128]; dO: [N,128] (any
-    float dtype, used in fp64).  Returns (dqhat, dkhat, dv), fp64 [N,128]."""
+    float dtype, used in fp64); O: optional forward output [N,128] that D is
+    taken from (default: the exact definition).  Returns (dqhat, dkhat, dv),
+    fp64 [N,128]."""
     qhat = np.ascontiguousarray(qhat, dtype=np.float32)
     khat = np.ascontiguousarray(khat, dtype=np.float32)
     v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
@@ -262,7 +265,11 @@ def attention_backward_head(qhat: np.ndarray, khat: np.ndarray, v_bits: np.ndarr
     if scale is None:
         scale = 1.0 / np.sqrt(128.0)
     dq, dk, dv = (np.empty((N, 128), np.float64) for _ in range(3))
-    lib().oracle_attention_backward_head(_p(qhat), _p(khat), _p(v_bits), _p(dO), N, float(scale),
+    op = None
+    if O is not None:
+        O = np.ascontiguousarray(O, dtype=np.float64)
+        op = _p(O)
+    lib().oracle_attention_backward_head(_p(qhat), _p(khat), _p(v_bits), _p(dO), op, N, float(scale),
                                          _p(dq), _p(dk), _p(dv))
     return dq, dk, dv
 
@@ -278,17 +285,19 @@ def ste_grads(dqhat: np.ndarray, dkhat: np.ndarray, flags: int = 0):
     return dq, dk
 
 
-def attention_backward(q_codes, q_scales, k_codes, k_scales, v_bits, dO, gq=1.0, gk=1.0, scale=None, flags=0):
+def attention_backward(q_codes, q_scales, k_codes, k_scales, v_bits, dO, gq=1.0, gk=1.0, scale=None, flags=0,
+                       O=None):
     """Whole training-time backward over [B,H,N,...] quantised Q/K, bf16 V and
     dO: attention gradients at the dequantised Q and K, then the straight-
-    through gradients of the bf16 Q and K inputs.  Returns (dq, dk, dv), fp64
-    [B,H,N,128]."""
+    through gradients of the bf16 Q and K inputs.  O: optional [B,H,N,128]
+    forward output D is taken from.  Returns (dq, dk, dv), fp64 [B,H,N,128]."""
     B, H, N = q_codes.shape[:3]
     out = [np.empty((B, H, N, 128), np.float64) for _ in range(3)]
     for b in range(B):
         for h in range(H):
             qh = dequant(q_codes[b, h], q_scales[b, h], gq)
             kh = dequant(k_codes[b, h], k_scales[b, h], gk)
-            dqh, dkh, out[2][b, h] = attention_backward_head(qh, kh, v_bits[b, h], dO[b, h], scale)
+            dqh, dkh, out[2][b, h] = attention_backward_head(qh, kh, v_bits[b, h], dO[b, h], scale,
+                                                             None if O is None else O[b, h])
             out[0][b, h], out[1][b, h] = ste_grads(dqh, dkh, flags)
     return tuple(out)

@@ -395,7 +395,8 @@ static double score_row(const float* q, const float* khat, int64_t N, double sca
 }
 
 void oracle_attention_backward_head(const float* qhat, const float* khat, const uint16_t* v, const double* dO,
-                                    int64_t N, double scale, double* dqhat, double* dkhat, double* dv) {
+                                    const double* O_in, int64_t N, double scale, double* dqhat, double* dkhat,
+                                    double* dv) {
     double* lse = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
     double* D = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
     /* pass over queries: lse_i, D_i = sum_j P_ij dP_ij, dQhat_i = scale sum_j dS_ij khat_j */
@@ -407,12 +408,15 @@ void oracle_attention_backward_head(const float* qhat, const float* khat, const 
             const double li = score_row(qhat + i * 128, khat, N, scale, s);
             const double* g = dO + i * 128;
             double Di = 0.0;
-            for (int64_t j = 0; j < N; ++j) {
-                const uint16_t* vv = v + j * 128;
-                double dp = 0.0;
-                for (int c = 0; c < 128; ++c) dp += g[c] * (double)oracle_bf16_to_f32(vv[c]);
-                s[j] = exp(s[j] - li) * dp; /* P_ij dP_ij */
-                Di += s[j];
+            if (O_in) { /* D from the given forward output: sum_c dO_ic O_ic */
+                for (int c = 0; c < 128; ++c) Di += g[c] * O_in[i * 128 + c];
+            } else {    /* the definition: sum_j P_ij dP_ij */
+                for (int64_t j = 0; j < N; ++j) {
+                    const uint16_t* vv = v + j * 128;
+                    double dp = 0.0;
+                    for (int c = 0; c < 128; ++c) dp += g[c] * (double)oracle_bf16_to_f32(vv[c]);
+                    Di += exp(s[j] - li) * dp;
+                }
             }
             lse[i] = li;
             D[i] = Di;

@@ -119,10 +119,13 @@ int oracle_num_threads(void);
  *   D_i = sum_j P_ij dP_ij, dS = P * (dP - D),
  *   dqhat = scale * dS khat, dkhat = scale * dS^T qhat, dv = P^T dO.
  * qhat, khat: fp32 [N,128]; v: bf16 bits [N,128]; dO: fp64 [N,128];
- * outputs fp64 [N,128]. */
+ * outputs fp64 [N,128].  O_in: NULL, or a forward output [N,128] from which
+ * D is taken instead (D_i = sum_c dO_ic O_in_ic, equal to the definition when
+ * O_in is the exact O): the backward's contract when the caller supplies the
+ * forward's stored output. */
 void oracle_attention_backward_head(const float* qhat, const float* khat, const uint16_t* v_bf16,
-                                    const double* dO, int64_t N, double scale, double* dqhat,
-                                    double* dkhat, double* dv);
+                                    const double* dO, const double* O_in, int64_t N, double scale,
+                                    double* dqhat, double* dkhat, double* dv);
 
 /* Straight-through estimator of the prologue for one head: the quantiser
  * passes gradients unchanged, the exact transforms are differentiated.

@@ -110,3 +110,20 @@ def test_strided_and_dynamic_validation_before_launch(fa):
         st = [good] * 4
         st[i] = bad
         assert bex(p, st[0], p, st[1], p, st[2], shape, 0.0, p, st[3], None, p, 1 << 20, None) == fa.ERR_INVALID_ARG
+
+
+def test_backward_validation_before_launch(fa):
+    S = fa.Shape
+    p = ctypes.c_void_p(4096)
+    f = fa.lib.fp4attn_backward
+    shape = S(1, 2, 128, 128)
+    wsb = fa.fp4attn_backward_workspace_bytes(1, 2, 128)
+    assert wsb >= 256 + 2 * 128 * 4 + 2 * 128 * 4 + 2 * 128 * 128 * 4
+    assert f(p, p, p, p, p, p, S(1, 2, 128, 64), 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_UNSUPPORTED
+    assert f(p, p, p, p, p, p, shape, 0.0, 0, p, p, p, p, wsb - 16, None) == fa.ERR_WORKSPACE
+    assert f(p, p, p, p, p, p, shape, 0.0, 8, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, p, p, p, p, shape, float("nan"), 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, p, p, p, None, shape, 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, p, p, p, p, shape, 0.0, 0, p, ctypes.c_void_p(4104), p, p, wsb, None) == fa.ERR_INVALID_ARG
+    d = fa.lib.fp4attn_dequant_bf16
+    assert d(p, ctypes.c_void_p(4100), None, shape, p, None) == fa.ERR_INVALID_ARG

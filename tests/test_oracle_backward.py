@@ -157,3 +157,17 @@ def test_attention_backward_over_quantised_heads():
         assert np.array_equal(dq[0, h], e) and np.array_equal(dk[0, h], f) and np.array_equal(dv[0, h], c)
     # the straight-through key gradient has zero column sums (the centring)
     assert np.abs(dk.sum(axis=2)).max() <= 1e-9 * np.abs(dk).max() * 96
+
+
+def test_backward_with_given_output_equals_definition_at_the_exact_output():
+    """D taken from a supplied forward output equals the definition when that
+    output is the exact O, and moves with it otherwise (the contract of a
+    backward that receives the stored forward output)."""
+    q, k, vb, v, dO = _head(90, seed=31, k_bias=1.0)
+    O, _ = oracle.attention_head(q, k, vb)
+    a = oracle.attention_backward_head(q, k, vb, dO)
+    b = oracle.attention_backward_head(q, k, vb, dO, O=O)
+    for x, y in zip(a, b):
+        assert np.allclose(x, y, rtol=1e-11, atol=1e-13 * np.abs(x).max())
+    c = oracle.attention_backward_head(q, k, vb, dO, O=O + 0.01)
+    assert not np.allclose(c[0], a[0], rtol=1e-6) and np.array_equal(c[2], a[2])
