@@ -44,7 +44,7 @@ namespace {
 
 constexpr int BR = 128;     // rows of the resident tile (queries or keys)
 constexpr int BS = 64;      // rows of a streamed stage (keys or queries)
-constexpr int STAGES = 3;
+constexpr int STAGES = 4;
 constexpr int THREADS = 192;
 constexpr int WARP_PRODUCER = 4;
 constexpr int WARP_MMA = 5;
@@ -470,6 +470,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         const float* lse_head = p.lse + (size_t)bh * N;
         const float* d_head = p.dsum + (size_t)bh * N;
+        // lse and D of the next stage are loaded one stage ahead, so their
+        // latency overlaps the wait for a free buffer
+        float nl[BS / 32], nd[BS / 32];
+        auto fetch = [&](int i) {
+#pragma unroll
+            for (int e = 0; e < BS / 32; ++e) {
+                const int qi = i * BS + lane + 32 * e;
+                nl[e] = (qi < N) ? lse_head[qi] * kLog2e : INFINITY;
+                nd[e] = (qi < N) ? d_head[qi] : 0.0f;
+            }
+        };
+        fetch(0);
         int issued = 0;
         for (int i = 0; i < T; ++i) {
             const int st = i % STAGES;
@@ -477,11 +489,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 !warp_wait(smem_u32(&sm.bar_q_empty[st]), ((i / STAGES) - 1) & 1, abort_flag, p.status, limit))
                 break;
 #pragma unroll
-            for (int e = lane; e < BS; e += 32) {
-                const int qi = i * BS + e;
-                sm.lse2[st][e] = (qi < N) ? lse_head[qi] * kLog2e : INFINITY;
-                sm.dsum[st][e] = (qi < N) ? d_head[qi] : 0.0f;
+            for (int e = 0; e < BS / 32; ++e) {
+                sm.lse2[st][lane + 32 * e] = nl[e];
+                sm.dsum[st][lane + 32 * e] = nd[e];
             }
+            if (i + 1 < T) fetch(i + 1);
             const uint32_t full = smem_u32(&sm.bar_q_full[st]);
             if (lane == 0) {
                 const int r0 = i * BS;

@@ -181,3 +181,29 @@ def test_backward_mid_workload_two_heads():
         _assert_close(dq[0, h], rq[0, 0], f"mid h{h} dq", tol=E2E_DQK)
         _assert_close(dk[0, h], rk[0, 0], f"mid h{h} dk", tol=E2E_DQK)
         _assert_close(dv[0, h], rv[0, 0], f"mid h{h} dv")
+
+
+@pytest.mark.parametrize("name,kw", [("N(0,1)", dict(seed=51)),
+                                     ("bias + outliers", dict(seed=52, k_offset_std=2.0, n_outliers=2,
+                                                              outlier_factor=20.0))])
+def test_fake_quant_forward_matches_the_fp4_kernel_within_1pct_of_quantisation_error(name, kw):
+    """The page's summary claim, checked between this library's kernels: the
+    fake-quantised forward (the BF16 kernel on the dequantised Q^ and K^, as a
+    training framework would run it) differs from the FP4 kernel by under 1% of
+    the FP4 kernel's own quantisation error (its distance to the BF16 kernel on
+    the unquantised Q and K)."""
+    w = synth.custom("fakeq", 1, 4, 4096, **kw)
+    d = synth.generate(w)
+    q, k, v = (d[t].cuda() for t in "qkv")
+    out = fa().fp4attn_quantize_qk(q, k)  # smoothing shifts each score row: softmax ignores it
+    o4, _ = fa().fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v,
+                                 workspace=out["workspace"])
+    qh = fa().fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])
+    kh = fa().fp4attn_dequant_bf16(out["k_codes"], out["k_scales"])
+    of, _ = fa().fp4attn_forward_bf16qk(qh, kh, v)
+    ob, _ = fa().fp4attn_forward_bf16qk(q, k, v)
+    assert fa().fp4attn_read_status(out["workspace"]) == 0
+    quant_err = torch.linalg.vector_norm((o4.float() - ob.float()))
+    fake_gap = torch.linalg.vector_norm((of.float() - o4.float()))
+    print(f"{name}: |fake - fp4| / |fp4 - bf16| = {float(fake_gap / quant_err):.4f}")
+    assert fake_gap <= 0.01 * quant_err
