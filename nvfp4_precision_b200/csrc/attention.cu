@@ -53,8 +53,10 @@ constexpr int WARP_PRODUCER = SOFTMAX_WARPS;
 constexpr int WARP_MMA = SOFTMAX_WARPS + 1;
 // Register split: three warps share each SM sub-partition's 16384 registers,
 // so the launch gets 168 per thread; the producer/MMA warpgroup gives most of
-// its share to the softmax warpgroups (2 x 128 x 232 + 128 x 40 = 384 x 168).
-constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 224, SUPPORT_REGS = 56;
+// its share to the softmax warpgroups (2 x 128 x 216 + 128 x 64 <= 384 x 168).
+// Measured: the softmax warps spill below 216; 64 for the producer and MMA
+// warps beats 56 (fewer spills there) and, oddly, 72.
+constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, SUPPORT_REGS = 64;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * SUPPORT_REGS <= FWD_THREADS * LAUNCH_REGS, "register split");
 static_assert((2 * SOFTMAX_REGS + SUPPORT_REGS) * 32 <= 16384, "registers of one SM sub-partition");
 // Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
