@@ -55,6 +55,7 @@ def test_quantize_validation_before_launch(fa):
     assert _q(fa, S(1, 1, 128, 64)) == fa.ERR_UNSUPPORTED          # D != 128
     assert _q(fa, S(1, -1, 128, 128)) == fa.ERR_INVALID_ARG        # negative size
     assert _q(fa, S(1, 1, 1 << 19, 128)) == fa.ERR_UNSUPPORTED     # N beyond the exact-sum range
+    assert _q(fa, S(1, 1, (1 << 18) + 1, 128)) == fa.ERR_UNSUPPORTED
     assert _q(fa, S(1, 1, 128, 128), flags=8) == fa.ERR_INVALID_ARG
     assert _q(fa, S(1, 1, 128, 128), ws=None) == fa.ERR_WORKSPACE
     assert _q(fa, S(1, 1, 128, 128), wsb=16) == fa.ERR_WORKSPACE
