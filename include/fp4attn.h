@@ -16,13 +16,18 @@
  *      channels under an fp32 per-tensor scale (unit by default);
  *   4. softmax(Q K^T * scale) V with Q K^T from the FP4 operands and P, V in
  *      BF16, non-causal, dense.
+ * Also here: the same attention with BF16 Q and K (the layers kept in BF16),
+ * an optional dynamic per-tensor scale (section "NVFP4 QAD": scaling to the
+ * largest value), and the training-time straight-through backward.
  * Details the pages leave open are fixed as follows: block scale amax/6,
  * round-to-nearest-even with saturation for both formats, Sylvester-ordered
  * Hadamard applied as seven fp32 butterfly stages of ascending stride followed
  * by one multiply by fp32(1/sqrt(128)), and an exact int64 fixed-point key sum
  * (2^-24 resolution) so the mean does not depend on summation order.
  *
- * Layouts (all tensors contiguous, row-major, head dim D = 128):
+ * Layouts (row-major, head dim D = 128; contiguous for the plain entry points,
+ * any strides for the bf16 tensors of the *_ex entry points, see
+ * fp4attn_strides):
  *   Q, K, V      bf16  [B, H, N, 128]
  *   codes        uint8 [B, H, N, 64]   element 2i in the low nibble of byte i;
  *                                      sign in bit 3 of each nibble
