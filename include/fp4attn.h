@@ -224,8 +224,14 @@ int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, 
  *   dq = c H dQ^, dk = c H (dK^ - mean_n dK^)   (c = 1/sqrt(128)).
  * P and dS are rounded to bf16 for the BF16 tensor-core products, which
  * accumulate in fp32; dq, dk, dv are bf16.
- *   qhat_dev, khat_dev : [B,H,N,128] bf16 dequantised Q and K (global scale
- *     included), e.g. from fp4attn_dequant_bf16.
+ *   qhat_dev, khat_dev : [B,H,N,128] bf16 unit-scale dequantised Q and K
+ *     (block scale x E2M1, exact in bf16): fp4attn_dequant_bf16 with a NULL
+ *     scale.
+ *   q_gscale_dev, k_gscale_dev : the forward's global scales (device fp32
+ *     scalars, finite and > 0), or NULL for 1.0.  Q^ = gQ * qhat and
+ *     K^ = gK * khat; the scales are applied as scalars (in the softmax scale
+ *     and the dQ^ / dK^ factors), never by rounding gQ * qhat to bf16, so the
+ *     backward's scores equal the forward's.
  *   v_dev, o_dev, do_dev : [B,H,N,128] bf16: V, the forward's O and dL/dO.
  *   lse_dev : [B,H,N] fp32 from the forward.
  *   softmax_scale : that of the forward (<= 0 selects 1/sqrt(128)).
@@ -234,13 +240,15 @@ int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, 
  *     K (the prologue's inputs) and V.
  *   workspace_dev : fp4attn_backward_workspace_bytes(s) bytes (status word
  *     first, so fp4attn_read_status works on it; about 512 bytes per row).
- * All tensors contiguous.  Device errors: FP4ATTN_ERR_TIMEOUT if an internal
+ * All tensors contiguous.  Device errors: FP4ATTN_ERR_RANGE for a bad global
+ * scale; FP4ATTN_ERR_TIMEOUT if an internal
  * wait ran out. */
 size_t fp4attn_backward_workspace_bytes(fp4attn_shape s);
-int fp4attn_backward(const void* qhat_dev, const void* khat_dev, const void* v_dev, const void* o_dev,
-                     const void* do_dev, const float* lse_dev, fp4attn_shape s, float softmax_scale,
-                     uint32_t flags, void* dq_dev, void* dk_dev, void* dv_dev, void* workspace_dev,
-                     size_t workspace_bytes, cudaStream_t stream);
+int fp4attn_backward(const void* qhat_dev, const void* khat_dev, const float* q_gscale_dev,
+                     const float* k_gscale_dev, const void* v_dev, const void* o_dev, const void* do_dev,
+                     const float* lse_dev, fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq_dev,
+                     void* dk_dev, void* dv_dev, void* workspace_dev, size_t workspace_bytes,
+                     cudaStream_t stream);
 
 /* Decode NVFP4 rows to bf16: out = bf16(fl(fl(g * s) * e2m1)), exact when
  * g = 1.  codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or

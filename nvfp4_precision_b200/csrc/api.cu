@@ -260,9 +260,10 @@ size_t fp4attn_backward_workspace_bytes(fp4attn_shape s) {
     return bws_bytes(bh, s.N > 0 ? s.N : 0);
 }
 
-int fp4attn_backward(const void* qhat, const void* khat, const void* v, const void* o, const void* dout,
-                     const float* lse, fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq, void* dk,
-                     void* dv, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const float* gk, const void* v,
+                     const void* o, const void* dout, const float* lse, fp4attn_shape s, float softmax_scale,
+                     uint32_t flags, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
     int st = check_shape(s);
     if (st != FP4ATTN_OK) return st;
     if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD)) return FP4ATTN_ERR_INVALID_ARG;
@@ -274,6 +275,7 @@ int fp4attn_backward(const void* qhat, const void* khat, const void* v, const vo
         for (const void* p : ptrs)
             if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
     }
+    if ((gq && ((uintptr_t)gq & 3)) || (gk && ((uintptr_t)gk & 3))) return FP4ATTN_ERR_INVALID_ARG;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int64_t BH = heads(s);
     cudaError_t e = cudaMemsetAsync(ws, 0, WS_STATUS_BYTES, stream);
@@ -282,6 +284,8 @@ int fp4attn_backward(const void* qhat, const void* khat, const void* v, const vo
     BwdArgs a;
     a.qhat = static_cast<const __nv_bfloat16*>(qhat);
     a.khat = static_cast<const __nv_bfloat16*>(khat);
+    a.gq = gq;
+    a.gk = gk;
     a.v = static_cast<const __nv_bfloat16*>(v);
     a.o = static_cast<const __nv_bfloat16*>(o);
     a.dout = static_cast<const __nv_bfloat16*>(dout);

@@ -5,9 +5,10 @@
 // student with 4-bit math on from the first step, and the summary list says
 // the training-time FP4 attention matches the inference kernel.  The forward
 // is the inference path itself (quantise, FP4 attention); the backward takes
-// the attention gradients at the dequantised Q^ and K^ (bf16, exact for a unit
-// global scale), passes them unchanged through the quantiser and
-// differentiates the exact transforms:
+// the attention gradients at the dequantised Q^ = gQ Q~ and K^ = gK K~, with
+// Q~, K~ the unit-scale values (scale x E2M1: exact in bf16) and the global
+// scales folded in as scalars, passes them unchanged through the quantiser
+// and differentiates the exact transforms:
 //   dS = P * (dP - D),  P = exp(scale Q^K^T - lse),  dP = dO V^T,
 //   D_i = sum_c dO_ic O_ic,
 //   dQ^ = scale dS K^,  dK^ = scale dS^T Q^,  dV = P^T dO,
@@ -114,6 +115,8 @@ struct BwdParams {
     int n_st;          // streamed stages of BS rows
     float scale;       // softmax scale
     float scale_log2;  // softmax scale * log2(e)
+    const float* gq;   // global scales of Q and K (device scalars, nullptr = 1)
+    const float* gk;
     const float* lse;  // [BH, N], natural log
     float* dsum;       // [BH, N]: D, written by bwd_q_kernel, read by bwd_kv_kernel
     const __nv_bfloat16* o;
@@ -310,7 +313,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             p.dsum[grow] = Dr;
             lse2 = p.lse[grow] * kLog2e;
         }
-        const float c = p.scale_log2;
+        const float gq = p.gq ? *p.gq : 1.0f, gk = p.gk ? *p.gk : 1.0f;
+        if (threadIdx.x == 0 && blockIdx.x == 0 && !(gq > 0.0f && gq < INFINITY && gk > 0.0f && gk < INFINITY))
+            atomicCAS(p.status, 0, (int)FP4ATTN_ERR_RANGE);
+        const float c = p.scale_log2 * gq * gk;  // S = scale gQ gK Q~ K~^T
+        const float dq_scale = p.scale * gk;     // dQ^ = scale dS K^ = scale gK dS K~
         bool ok = true;
         for (int j = 0; j < T; ++j) {
             const int b = j & 1;
@@ -352,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tmem_ld32(tmem + lane_base + TM_ACC0 + 32u * q, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[32 * q + e] = __uint_as_float(r[e]) * p.scale;
+                for (int e = 0; e < 32; ++e) x[32 * q + e] = __uint_as_float(r[e]) * dq_scale;
             }
             if (p.hadamard) {
                 fwht128(x);
@@ -588,7 +595,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int row = 32 * warp + lane;  // key row of the tile
         const int kn = k0 + row;
         const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        const float c = p.scale_log2;
+        const float gq = p.gq ? *p.gq : 1.0f, gk = p.gk ? *p.gk : 1.0f;
+        const float c = p.scale_log2 * gq * gk;  // S^T = scale gQ gK K~ Q~^T
+        const float dk_scale = p.scale * gq;     // dK^ = scale dS^T Q^ = scale gQ dS^T Q~
         bool ok = true;
         for (int i = 0; i < T; ++i) {
             const int b = i & 1;
@@ -660,7 +669,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tmem_ld32(tmem + lane_base + TM_ACC1 + 32u * q, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[32 * q + e] = valid ? __uint_as_float(r[e]) * p.scale : 0.0f;
+                for (int e = 0; e < 32; ++e) x[32 * q + e] = valid ? __uint_as_float(r[e]) * dk_scale : 0.0f;
             }
             if (valid) {
                 float4* dst = reinterpret_cast<float4*>(p.dk_acc + grow * 128);
@@ -771,6 +780,8 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     p.n_st = (a.N + BS - 1) / BS;
     p.scale = a.softmax_scale > 0.0f ? a.softmax_scale : 0.08838834764831845f;
     p.scale_log2 = p.scale * kLog2e;
+    p.gq = a.gq;
+    p.gk = a.gk;
     p.lse = a.lse;
     p.dsum = a.dsum;
     p.o = a.o;

@@ -114,8 +114,10 @@ inline size_t bws_dk_offset(int64_t BH, int64_t N) {
 inline size_t bws_bytes(int64_t BH, int64_t N) { return bws_dk_offset(BH, N) + bws_align((size_t)(BH * N) * D * 4); }
 
 struct BwdArgs {
-    const __nv_bfloat16* qhat;  // dequantised Q and K, [B,H,N,128] contiguous
+    const __nv_bfloat16* qhat;  // unit-scale dequantised Q and K, [B,H,N,128] contiguous
     const __nv_bfloat16* khat;
+    const float* gq;            // global scales (device scalars) or nullptr for 1
+    const float* gk;
     const __nv_bfloat16* v;
     const __nv_bfloat16* o;
     const __nv_bfloat16* dout;

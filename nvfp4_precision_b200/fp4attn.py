@@ -81,7 +81,8 @@ def _load():
     L.fp4attn_backward_workspace_bytes.restype = ctypes.c_size_t
     L.fp4attn_backward_workspace_bytes.argtypes = [Shape]
     L.fp4attn_backward.restype = ctypes.c_int
-    L.fp4attn_backward.argtypes = [P, P, P, P, P, P, Shape, ctypes.c_float, U32, P, P, P, P, ctypes.c_size_t, P]
+    L.fp4attn_backward.argtypes = [P, P, P, P, P, P, P, P, Shape, ctypes.c_float, U32, P, P, P, P, ctypes.c_size_t,
+                                   P]
     L.fp4attn_dequant.restype = ctypes.c_int
     L.fp4attn_dequant.argtypes = [P, P, P, Shape, P, P]
     L.fp4attn_read_status.restype = ctypes.c_int
@@ -284,11 +285,13 @@ def fp4attn_backward_workspace_bytes(B: int, H: int, N: int, D: int = 128) -> in
 
 
 def fp4attn_backward(qhat, khat, v, o, dout, lse, softmax_scale: float = 0.0, flags: int = 0,
-                     workspace: Optional[torch.Tensor] = None, stream=None):
+                     workspace: Optional[torch.Tensor] = None, stream=None, q_gscale: Optional[torch.Tensor] = None,
+                     k_gscale: Optional[torch.Tensor] = None):
     """Straight-through backward of the FP4 attention (see include/fp4attn.h):
-    bf16 [B,H,N,128] dequantised Q^, K^, V, the forward's O, dL/dO, fp32 lse
-    [B,H,N].  Returns (dq, dk, dv, workspace), bf16 gradients of the bf16 Q,
-    K, V inputs of the forward."""
+    bf16 [B,H,N,128] unit-scale dequantised Q~, K~ (fp4attn_dequant_bf16 with
+    no scale), V, the forward's O, dL/dO, fp32 lse [B,H,N], and the forward's
+    global scales (device scalars, None for 1).  Returns (dq, dk, dv,
+    workspace), bf16 gradients of the bf16 Q, K, V inputs of the forward."""
     for t in (qhat, khat, v, o, dout):
         assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == v.shape
     assert lse.dtype == torch.float32 and lse.is_contiguous()
@@ -296,7 +299,8 @@ def fp4attn_backward(qhat, khat, v, o, dout, lse, softmax_scale: float = 0.0, fl
     if workspace is None:
         workspace = torch.empty(fp4attn_backward_workspace_bytes(B, H, N), dtype=torch.uint8, device=v.device)
     dq, dk, dv = (torch.empty((B, H, N, D), dtype=torch.bfloat16, device=v.device) for _ in range(3))
-    rc = lib.fp4attn_backward(_ptr(qhat), _ptr(khat), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), Shape(B, H, N, D),
+    rc = lib.fp4attn_backward(_ptr(qhat), _ptr(khat), _ptr(q_gscale), _ptr(k_gscale), _ptr(v), _ptr(o), _ptr(dout),
+                              _ptr(lse), Shape(B, H, N, D),
                               float(softmax_scale), int(flags), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                               workspace.numel(), _stream(stream))
     _check(rc, "fp4attn_backward")
@@ -309,36 +313,38 @@ class FP4AttentionSTE(torch.autograd.Function):
     status words of both halves are checked on the host."""
 
     @staticmethod
-    def forward(ctx, q, k, v, softmax_scale=0.0, flags=0):
+    def forward(ctx, q, k, v, softmax_scale=0.0, flags=0, dynamic_gscale=False):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        out = fp4attn_quantize_qk(q, k, flags=flags, k_mean=False)
-        o, lse = fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v,
+        out = fp4attn_quantize_qk(q, k, flags=flags, k_mean=False, dynamic_gscale=dynamic_gscale)
+        gq, gk = out.get("q_gscale"), out.get("k_gscale")
+        o, lse = fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, gq, gk,
                                  softmax_scale=softmax_scale, want_lse=True, workspace=out["workspace"])
-        qhat = fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])
+        qhat = fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])  # unit scale: exact in bf16
         khat = fp4attn_dequant_bf16(out["k_codes"], out["k_scales"])
         st = fp4attn_read_status(out["workspace"])
         if st != OK:
             raise Fp4AttnError(st, "FP4AttentionSTE.forward (device)")
-        ctx.save_for_backward(qhat, khat, v, o, lse)
+        ctx.save_for_backward(qhat, khat, v, o, lse, gq, gk)
         ctx.softmax_scale, ctx.flags = softmax_scale, flags
         return o
 
     @staticmethod
     def backward(ctx, do):
-        qhat, khat, v, o, lse = ctx.saved_tensors
+        qhat, khat, v, o, lse, gq, gk = ctx.saved_tensors
         dq, dk, dv, ws = fp4attn_backward(qhat, khat, v, o, do.contiguous().to(torch.bfloat16), lse,
-                                          ctx.softmax_scale, ctx.flags)
+                                          ctx.softmax_scale, ctx.flags, q_gscale=gq, k_gscale=gk)
         st = fp4attn_read_status(ws)
         if st != OK:
             raise Fp4AttnError(st, "FP4AttentionSTE.backward (device)")
-        return dq, dk, dv, None, None
+        return dq, dk, dv, None, None, None
 
 
 def fp4_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, softmax_scale: float = 0.0,
-                  flags: int = 0) -> torch.Tensor:
+                  flags: int = 0, dynamic_gscale: bool = False) -> torch.Tensor:
     """Differentiable FP4 attention of bf16 [B,H,N,128] Q, K, V (fake
-    quantisation with a straight-through backward)."""
-    return FP4AttentionSTE.apply(q, k, v, softmax_scale, flags)
+    quantisation with a straight-through backward); dynamic_gscale selects the
+    amax-derived per-tensor scales."""
+    return FP4AttentionSTE.apply(q, k, v, softmax_scale, flags, dynamic_gscale)
 
 
 def fp4attn_read_status(workspace: torch.Tensor, stream=None) -> int:

@@ -120,11 +120,14 @@ def test_backward_validation_before_launch(fa):
     shape = S(1, 2, 128, 128)
     wsb = fa.fp4attn_backward_workspace_bytes(1, 2, 128)
     assert wsb >= 256 + 2 * 128 * 4 + 2 * 128 * 4 + 2 * 128 * 128 * 4
-    assert f(p, p, p, p, p, p, S(1, 2, 128, 64), 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_UNSUPPORTED
-    assert f(p, p, p, p, p, p, shape, 0.0, 0, p, p, p, p, wsb - 16, None) == fa.ERR_WORKSPACE
-    assert f(p, p, p, p, p, p, shape, 0.0, 8, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
-    assert f(p, p, p, p, p, p, shape, float("nan"), 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
-    assert f(p, p, p, p, p, None, shape, 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
-    assert f(p, p, p, p, p, p, shape, 0.0, 0, p, ctypes.c_void_p(4104), p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, None, None, p, p, p, p, S(1, 2, 128, 64), 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_UNSUPPORTED
+    assert f(p, p, None, None, p, p, p, p, shape, 0.0, 0, p, p, p, p, wsb - 16, None) == fa.ERR_WORKSPACE
+    assert f(p, p, None, None, p, p, p, p, shape, 0.0, 8, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, None, None, p, p, p, p, shape, float("nan"), 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, None, None, p, p, p, None, shape, 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
+    assert f(p, p, None, None, p, p, p, p, shape, 0.0, 0, p, ctypes.c_void_p(4104), p, p, wsb, None) \
+        == fa.ERR_INVALID_ARG
+    assert f(p, p, ctypes.c_void_p(4098), None, p, p, p, p, shape, 0.0, 0, p, p, p, p, wsb, None) \
+        == fa.ERR_INVALID_ARG
     d = fa.lib.fp4attn_dequant_bf16
     assert d(p, ctypes.c_void_p(4100), None, shape, p, None) == fa.ERR_INVALID_ARG

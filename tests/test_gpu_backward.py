@@ -207,3 +207,58 @@ def test_fake_quant_forward_matches_the_fp4_kernel_within_1pct_of_quantisation_e
     fake_gap = torch.linalg.vector_norm((of.float() - o4.float()))
     print(f"{name}: |fake - fp4| / |fp4 - bf16| = {float(fake_gap / quant_err):.4f}")
     assert fake_gap <= 0.01 * quant_err
+
+
+def test_autograd_with_dynamic_scales_and_flags():
+    """fp4_attention with the dynamic per-tensor scales and each transform off:
+    gradients against the oracle's (same g, end-to-end bounds).  The backward
+    gets the unit-scale Q~, K~ (exact in bf16) and g as scalars: rounding
+    g * Q~ to bf16 instead would move the scores of these outlier-heavy keys
+    (lse up to about 360) by tenths of a unit and the gradients by over 10%."""
+    w = synth.custom("bwd_dyn", 1, 2, 400, seed=91, k_offset_std=2.0, n_outliers=2, outlier_factor=20.0)
+    d = synth.generate(w)
+    dO = _dout((1, 2, 400, 128), seed=11)
+    for flags in (0, 3):
+        q, k, v = (d[t].cuda().requires_grad_(True) for t in "qkv")
+        o = fa().fp4_attention(q, k, v, flags=flags, dynamic_gscale=True)
+        o.backward(dO.cuda())
+        ref = oracle.quantize_qk(synth.bf16_bits(d["q"]), synth.bf16_bits(d["k"]), flags=flags, dynamic=True)
+        rq, rk, rv = oracle.attention_backward(ref["q_codes"], ref["q_scales"], ref["k_codes"], ref["k_scales"],
+                                               synth.bf16_bits(d["v"]), dO.double().numpy(), float(ref["gq"]),
+                                               float(ref["gk"]), flags=flags)
+        for h in range(2):
+            _assert_close(q.grad[0, h].float().cpu().numpy(), rq[0, h], f"dyn flags{flags} h{h} dq", tol=E2E_DQK)
+            _assert_close(k.grad[0, h].float().cpu().numpy(), rk[0, h], f"dyn flags{flags} h{h} dk", tol=E2E_DQK)
+            _assert_close(v.grad[0, h].float().cpu().numpy(), rv[0, h], f"dyn flags{flags} h{h} dv")
+
+
+def test_backward_kernel_parity_with_global_scales():
+    """Static global scales gQ = 0.37, gK = 1.9: the backward gets the unit-scale
+    Q~, K~ (exact in bf16) and the scales as scalars; same inputs on both sides
+    (the oracle's O rounded to bf16 and its lse), tight bounds."""
+    gq, gk = 0.37, 1.9
+    w = synth.custom("bwd_g", 1, 2, 333, seed=93, k_offset_std=2.0, n_outliers=2, outlier_factor=20.0)
+    d = synth.generate(w)
+    dO = _dout((1, 2, 333, 128), seed=13)
+    vb = synth.bf16_bits(d["v"])
+    codes = oracle.quantize_qk(synth.bf16_bits(d["q"]), synth.bf16_bits(d["k"]), gq, gk)
+    O = np.empty((1, 2, 333, 128))
+    L = np.empty((1, 2, 333))
+    for h in range(2):
+        O[0, h], L[0, h] = oracle.attention_head(oracle.dequant(codes["q_codes"][0, h], codes["q_scales"][0, h], gq),
+                                                 oracle.dequant(codes["k_codes"][0, h], codes["k_scales"][0, h], gk),
+                                                 vb[0, h])
+    o_bf = _bf16(O)
+    qt = _bf16(oracle.dequant(codes["q_codes"], codes["q_scales"])).cuda()
+    kt = _bf16(oracle.dequant(codes["k_codes"], codes["k_scales"])).cuda()
+    g = lambda x: torch.tensor([x], dtype=torch.float32, device="cuda")
+    dq, dk, dv, ws = fa().fp4attn_backward(qt, kt, d["v"].cuda(), o_bf.cuda(), dO.cuda(),
+                                           torch.from_numpy(L.astype(np.float32)).cuda(), q_gscale=g(gq),
+                                           k_gscale=g(gk))
+    assert fa().fp4attn_read_status(ws) == 0
+    rq, rk, rv = oracle.attention_backward(codes["q_codes"], codes["q_scales"], codes["k_codes"], codes["k_scales"],
+                                           vb, dO.double().numpy(), gq, gk, O=o_bf.double().numpy())
+    for h in range(2):
+        _assert_close(dq[0, h].float().cpu().numpy(), rq[0, h], f"g h{h} dq")
+        _assert_close(dk[0, h].float().cpu().numpy(), rk[0, h], f"g h{h} dk")
+        _assert_close(dv[0, h].float().cpu().numpy(), rv[0, h], f"g h{h} dv")
