@@ -250,6 +250,17 @@ int fp4attn_backward(const void* qhat_dev, const void* khat_dev, const float* q_
                      void* dk_dev, void* dv_dev, void* workspace_dev, size_t workspace_bytes,
                      cudaStream_t stream);
 
+/* fp4attn_backward with V, O, dO and the outputs dq, dk, dv in one layout of
+ * any element strides (fp4attn_strides; e.g. [B,N,H,128] as a QKV projection
+ * writes them); qhat, khat and lse stay contiguous (the library's own
+ * outputs).  The outputs' rows must not overlap one another or any input.
+ * Errors as for fp4attn_backward; FP4ATTN_ERR_INVALID_ARG for a bad stride. */
+int fp4attn_backward_ex(const void* qhat_dev, const void* khat_dev, const float* q_gscale_dev,
+                        const float* k_gscale_dev, const void* v_dev, const void* o_dev, const void* do_dev,
+                        fp4attn_strides io_strides, const float* lse_dev, fp4attn_shape s, float softmax_scale,
+                        uint32_t flags, void* dq_dev, void* dk_dev, void* dv_dev, void* workspace_dev,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 /* Decode NVFP4 rows to bf16: out = bf16(fl(fl(g * s) * e2m1)), exact when
  * g = 1.  codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or
  * NULL, out_dev bf16 [rows,128], rows = B*H*N of s. */

@@ -260,10 +260,10 @@ size_t fp4attn_backward_workspace_bytes(fp4attn_shape s) {
     return bws_bytes(bh, s.N > 0 ? s.N : 0);
 }
 
-int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const float* gk, const void* v,
-                     const void* o, const void* dout, const float* lse, fp4attn_shape s, float softmax_scale,
-                     uint32_t flags, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                     cudaStream_t stream) {
+int fp4attn_backward_ex(const void* qhat, const void* khat, const float* gq, const float* gk, const void* v,
+                        const void* o, const void* dout, fp4attn_strides io_strides, const float* lse,
+                        fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq, void* dk, void* dv,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     int st = check_shape(s);
     if (st != FP4ATTN_OK) return st;
     if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD)) return FP4ATTN_ERR_INVALID_ARG;
@@ -276,6 +276,8 @@ int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const 
             if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
     }
     if ((gq && ((uintptr_t)gq & 3)) || (gk && ((uintptr_t)gk & 3))) return FP4ATTN_ERR_INVALID_ARG;
+    Strides io{};
+    if (!empty(s) && !normalise_strides(s, io_strides, &io)) return FP4ATTN_ERR_INVALID_ARG;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int64_t BH = heads(s);
     cudaError_t e = cudaMemsetAsync(ws, 0, WS_STATUS_BYTES, stream);
@@ -289,6 +291,7 @@ int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const 
     a.v = static_cast<const __nv_bfloat16*>(v);
     a.o = static_cast<const __nv_bfloat16*>(o);
     a.dout = static_cast<const __nv_bfloat16*>(dout);
+    a.io = io;
     a.lse = lse;
     a.BH = (int)BH;
     a.H = s.H;
@@ -306,6 +309,14 @@ int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const 
     st = launch_backward(a, stream);
     if (st != FP4ATTN_OK) (void)cudaGetLastError();
     return st;
+}
+
+int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const float* gk, const void* v,
+                     const void* o, const void* dout, const float* lse, fp4attn_shape s, float softmax_scale,
+                     uint32_t flags, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
+    return fp4attn_backward_ex(qhat, khat, gq, gk, v, o, dout, contiguous(s), lse, s, softmax_scale, flags, dq, dk,
+                               dv, workspace, workspace_bytes, stream);
 }
 
 int fp4attn_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s, void* out,

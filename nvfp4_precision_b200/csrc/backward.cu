@@ -95,6 +95,12 @@ __device__ __forceinline__ uint64_t mn_desc(const uint8_t* tile, uint32_t panel)
 }
 constexpr uint64_t MN_KSTEP = 2048 >> 4;
 
+// Element offset of row n of head bh in a [B,H,N,128] tensor with strides (sb, sh, sn).
+__device__ __forceinline__ long long row_offset(int bh, int H, int n, long long sb, long long sh, long long sn) {
+    const int b = bh / H, h = bh - b * H;
+    return b * sb + h * sh + (long long)n * sn;
+}
+
 // In-register Walsh-Hadamard transform of 128 values (Sylvester order).
 __device__ __forceinline__ void fwht128(float* x) {
 #pragma unroll
@@ -121,8 +127,9 @@ struct BwdParams {
     float* dsum;       // [BH, N]: D, written by bwd_q_kernel, read by bwd_kv_kernel
     const __nv_bfloat16* o;
     const __nv_bfloat16* dout;
-    __nv_bfloat16* dq;  // [BH, N, 128]
+    __nv_bfloat16* dq;  // [B, H, N, 128], element strides io (as o, dout, dv)
     __nv_bfloat16* dv;
+    long long io_sb, io_sh, io_sn;
     float* dk_acc;      // [BH, N, 128] fp32: scale * dK^
     float* partial;     // [BH, key tiles * 4, 128] fp32: column sums of scale * dK^ per warp
     bool hadamard;
@@ -297,8 +304,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         // rows past N get p = 0 (lse = +inf) and D = 0
         float Dr = 0.0f, lse2 = INFINITY;
         if (n < N) {
-            const uint4* po = reinterpret_cast<const uint4*>(p.o + grow * 128);
-            const uint4* pd = reinterpret_cast<const uint4*>(p.dout + grow * 128);
+            const long long io = row_offset(bh, p.H, n, p.io_sb, p.io_sh, p.io_sn);
+            const uint4* po = reinterpret_cast<const uint4*>(p.o + io);
+            const uint4* pd = reinterpret_cast<const uint4*>(p.dout + io);
             float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll 4
             for (int c = 0; c < 16; ++c) {
@@ -368,7 +376,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int e = 0; e < 128; ++e) x[e] *= h;
             }
             if (n < N) {
-                uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * 128);
+                uint4* dst = reinterpret_cast<uint4*>(p.dq + row_offset(bh, p.H, n, p.io_sb, p.io_sh, p.io_sn));
 #pragma unroll
                 for (int v = 0; v < 16; ++v)
                     dst[v] = make_uint4(pack_bf16x2(x[8 * v], x[8 * v + 1]), pack_bf16x2(x[8 * v + 2], x[8 * v + 3]),
@@ -651,7 +659,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tmem_ld32(tmem + lane_base + TM_ACC0 + 32u * q, r);
                 tmem_wait_ld();
                 if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.dv + grow * 128 + 32 * q);
+                    uint4* dst = reinterpret_cast<uint4*>(p.dv + row_offset(bh, p.H, kn, p.io_sb, p.io_sh, p.io_sn) +
+                                                          32 * q);
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
                         dst[v] = make_uint4(
@@ -707,8 +716,9 @@ __global__ void __launch_bounds__(128) colsum_kernel(const float* __restrict__ p
 // holds channels 4l .. 4l+3; butterfly strides 1 and 2 stay in the lane,
 // strides 4 .. 64 pair lanes l and l ^ (stride / 4).
 __global__ void __launch_bounds__(256) ste_k_kernel(const float* __restrict__ dk_acc, const float* __restrict__ colsum,
-                                                    int N, int64_t rows, bool smooth, bool hadamard,
-                                                    __nv_bfloat16* __restrict__ dk) {
+                                                    int N, int H, int64_t rows, bool smooth, bool hadamard,
+                                                    __nv_bfloat16* __restrict__ dk, long long sb, long long sh,
+                                                    long long sn) {
     const int lane = threadIdx.x & 31;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const float nf = (float)N;
@@ -741,14 +751,16 @@ __global__ void __launch_bounds__(256) ste_k_kernel(const float* __restrict__ dk
 #pragma unroll
             for (int e = 0; e < 4; ++e) x[e] *= h;
         }
-        reinterpret_cast<uint2*>(dk + r * 128)[lane] = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+        const int bh = (int)(r / N), n = (int)(r - (int64_t)bh * N);
+        reinterpret_cast<uint2*>(dk + row_offset(bh, H, n, sb, sh, sn))[lane] =
+            make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
     }
 }
 
-// [B][H][N][128 bf16], contiguous: 128B-swizzled boxes of 64 channels x
-// box_rows rows of one head (x is 0 or 64: 16-byte aligned).
-bool make_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, uint32_t box_rows) {
-    const Strides st = contiguous_strides(H, N);
+// [B][H][N][128 bf16] with element strides st (multiples of 8): 128B-swizzled
+// boxes of 64 channels x box_rows rows of one head (x is 0 or 64: 16-byte
+// aligned).
+bool make_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, uint32_t box_rows, Strides st) {
     const uint64_t dims[4] = {128, (uint64_t)N, (uint64_t)H, (uint64_t)B};
     const uint64_t strides[3] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
     const uint32_t box[4] = {64, box_rows, 1, 1};
@@ -762,10 +774,11 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     const int B = a.BH / a.H;
     CUtensorMap q_r, do_r, k_s, v_s, k_r, v_r, q_s, do_s;
-    if (!make_map(&q_r, a.qhat, B, a.H, a.N, BR) || !make_map(&do_r, a.dout, B, a.H, a.N, BR) ||
-        !make_map(&k_s, a.khat, B, a.H, a.N, BS) || !make_map(&v_s, a.v, B, a.H, a.N, BS) ||
-        !make_map(&k_r, a.khat, B, a.H, a.N, BR) || !make_map(&v_r, a.v, B, a.H, a.N, BR) ||
-        !make_map(&q_s, a.qhat, B, a.H, a.N, BS) || !make_map(&do_s, a.dout, B, a.H, a.N, BS))
+    const Strides cs = contiguous_strides(a.H, a.N);  // Q~, K~: the library's own contiguous tensors
+    if (!make_map(&q_r, a.qhat, B, a.H, a.N, BR, cs) || !make_map(&do_r, a.dout, B, a.H, a.N, BR, a.io) ||
+        !make_map(&k_s, a.khat, B, a.H, a.N, BS, cs) || !make_map(&v_s, a.v, B, a.H, a.N, BS, a.io) ||
+        !make_map(&k_r, a.khat, B, a.H, a.N, BR, cs) || !make_map(&v_r, a.v, B, a.H, a.N, BR, a.io) ||
+        !make_map(&q_s, a.qhat, B, a.H, a.N, BS, cs) || !make_map(&do_s, a.dout, B, a.H, a.N, BS, a.io))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(QSmem) + 1024 <= 227 * 1024, "shared memory budget");
     static_assert(sizeof(KVSmem) + 1024 <= 227 * 1024, "shared memory budget");
@@ -788,6 +801,9 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     p.dout = a.dout;
     p.dq = a.dq;
     p.dv = a.dv;
+    p.io_sb = a.io.b;
+    p.io_sh = a.io.h;
+    p.io_sn = a.io.n;
     p.dk_acc = a.dk_acc;
     p.partial = a.partial;
     p.hadamard = !(a.flags & FP4ATTN_NO_HADAMARD);
@@ -805,8 +821,8 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     const int64_t rows = (int64_t)a.BH * a.N;
     const int64_t want = (rows + 7) / 8;  // 8 warps per block, one row each
     const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
-    ste_k_kernel<<<blocks, 256, 0, stream>>>(a.dk_acc, a.colsum, a.N, rows, !(a.flags & FP4ATTN_NO_SMOOTH_K),
-                                             p.hadamard, a.dk);
+    ste_k_kernel<<<blocks, 256, 0, stream>>>(a.dk_acc, a.colsum, a.N, a.H, rows, !(a.flags & FP4ATTN_NO_SMOOTH_K),
+                                             p.hadamard, a.dk, a.io.b, a.io.h, a.io.n);
     return cudaGetLastError() == cudaSuccess ? FP4ATTN_OK : FP4ATTN_ERR_CUDA;
 }
 

@@ -121,6 +121,7 @@ struct BwdArgs {
     const __nv_bfloat16* v;
     const __nv_bfloat16* o;
     const __nv_bfloat16* dout;
+    Strides io;        // element strides of v, o, dout, dq, dk, dv
     const float* lse;  // [B,H,N]
     int BH, H, N;
     float softmax_scale;

@@ -30,7 +30,8 @@ DYNAMIC_GSCALE = 4
 EXPORTS = (
     "fp4attn_workspace_bytes", "fp4attn_quantize_qk", "fp4attn_quantize_qk_ex", "fp4attn_quantize_qk_noalloc",
     "fp4attn_forward", "fp4attn_forward_ex", "fp4attn_forward_bf16qk", "fp4attn_forward_bf16qk_ex",
-    "fp4attn_dequant", "fp4attn_dequant_bf16", "fp4attn_backward", "fp4attn_backward_workspace_bytes",
+    "fp4attn_dequant", "fp4attn_dequant_bf16", "fp4attn_backward", "fp4attn_backward_ex",
+    "fp4attn_backward_workspace_bytes",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
 )
@@ -83,6 +84,9 @@ def _load():
     L.fp4attn_backward.restype = ctypes.c_int
     L.fp4attn_backward.argtypes = [P, P, P, P, P, P, P, P, Shape, ctypes.c_float, U32, P, P, P, P, ctypes.c_size_t,
                                    P]
+    L.fp4attn_backward_ex.restype = ctypes.c_int
+    L.fp4attn_backward_ex.argtypes = [P, P, P, P, P, P, P, Strides, P, Shape, ctypes.c_float, U32, P, P, P, P,
+                                      ctypes.c_size_t, P]
     L.fp4attn_dequant.restype = ctypes.c_int
     L.fp4attn_dequant.argtypes = [P, P, P, Shape, P, P]
     L.fp4attn_read_status.restype = ctypes.c_int
@@ -289,21 +293,28 @@ def fp4attn_backward(qhat, khat, v, o, dout, lse, softmax_scale: float = 0.0, fl
                      k_gscale: Optional[torch.Tensor] = None):
     """Straight-through backward of the FP4 attention (see include/fp4attn.h):
     bf16 [B,H,N,128] unit-scale dequantised Q~, K~ (fp4attn_dequant_bf16 with
-    no scale), V, the forward's O, dL/dO, fp32 lse [B,H,N], and the forward's
-    global scales (device scalars, None for 1).  Returns (dq, dk, dv,
-    workspace), bf16 gradients of the bf16 Q, K, V inputs of the forward."""
-    for t in (qhat, khat, v, o, dout):
+    no scale, contiguous), V, the forward's O, dL/dO (one layout of any
+    strides with contiguous channels, e.g. views of [B,N,H,128] tensors),
+    fp32 lse [B,H,N], and the forward's global scales (device scalars, None
+    for 1).  Returns (dq, dk, dv, workspace): bf16 gradients of the bf16 Q, K,
+    V inputs of the forward, in the layout of V."""
+    for t in (qhat, khat):
         assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == v.shape
+    st = strides_of(v)
+    for t in (o, dout):
+        assert t.dtype == torch.bfloat16 and t.shape == v.shape and t.stride() == v.stride(), \
+            "v, o and dout must share one layout"
+    assert v.dtype == torch.bfloat16
     assert lse.dtype == torch.float32 and lse.is_contiguous()
     B, H, N, D = v.shape
     if workspace is None:
         workspace = torch.empty(fp4attn_backward_workspace_bytes(B, H, N), dtype=torch.uint8, device=v.device)
-    dq, dk, dv = (torch.empty((B, H, N, D), dtype=torch.bfloat16, device=v.device) for _ in range(3))
-    rc = lib.fp4attn_backward(_ptr(qhat), _ptr(khat), _ptr(q_gscale), _ptr(k_gscale), _ptr(v), _ptr(o), _ptr(dout),
-                              _ptr(lse), Shape(B, H, N, D),
-                              float(softmax_scale), int(flags), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
-                              workspace.numel(), _stream(stream))
-    _check(rc, "fp4attn_backward")
+    dq, dk, dv = (torch.empty_strided(v.shape, v.stride(), dtype=torch.bfloat16, device=v.device) for _ in range(3))
+    rc = lib.fp4attn_backward_ex(_ptr(qhat), _ptr(khat), _ptr(q_gscale), _ptr(k_gscale), _ptr(v), _ptr(o),
+                                 _ptr(dout), st, _ptr(lse), Shape(B, H, N, D),
+                                 float(softmax_scale), int(flags), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+    _check(rc, "fp4attn_backward_ex")
     return dq, dk, dv, workspace
 
 
@@ -314,11 +325,14 @@ class FP4AttentionSTE(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, softmax_scale=0.0, flags=0, dynamic_gscale=False):
-        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        # any layout with contiguous channels is used as it is (no copies);
+        # O is allocated in V's layout, which the backward then uses throughout
+        q, k, v = (t if t.stride(3) == 1 and t.stride(0) > 0 else t.contiguous() for t in (q, k, v))
         out = fp4attn_quantize_qk(q, k, flags=flags, k_mean=False, dynamic_gscale=dynamic_gscale)
         gq, gk = out.get("q_gscale"), out.get("k_gscale")
+        o = torch.empty_strided(v.shape, v.stride(), dtype=torch.bfloat16, device=v.device)
         o, lse = fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, gq, gk,
-                                 softmax_scale=softmax_scale, want_lse=True, workspace=out["workspace"])
+                                 softmax_scale=softmax_scale, o=o, want_lse=True, workspace=out["workspace"])
         qhat = fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])  # unit scale: exact in bf16
         khat = fp4attn_dequant_bf16(out["k_codes"], out["k_scales"])
         st = fp4attn_read_status(out["workspace"])
@@ -331,8 +345,11 @@ class FP4AttentionSTE(torch.autograd.Function):
     @staticmethod
     def backward(ctx, do):
         qhat, khat, v, o, lse, gq, gk = ctx.saved_tensors
-        dq, dk, dv, ws = fp4attn_backward(qhat, khat, v, o, do.contiguous().to(torch.bfloat16), lse,
-                                          ctx.softmax_scale, ctx.flags, q_gscale=gq, k_gscale=gk)
+        do = do.to(torch.bfloat16)
+        if do.stride() != v.stride():
+            do = torch.empty_strided(v.shape, v.stride(), dtype=torch.bfloat16, device=v.device).copy_(do)
+        dq, dk, dv, ws = fp4attn_backward(qhat, khat, v, o, do, lse, ctx.softmax_scale, ctx.flags,
+                                          q_gscale=gq, k_gscale=gk)
         st = fp4attn_read_status(ws)
         if st != OK:
             raise Fp4AttnError(st, "FP4AttentionSTE.backward (device)")

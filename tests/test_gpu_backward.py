@@ -262,3 +262,26 @@ def test_backward_kernel_parity_with_global_scales():
         _assert_close(dq[0, h].float().cpu().numpy(), rq[0, h], f"g h{h} dq")
         _assert_close(dk[0, h].float().cpu().numpy(), rk[0, h], f"g h{h} dk")
         _assert_close(dv[0, h].float().cpu().numpy(), rv[0, h], f"g h{h} dv")
+
+
+def test_autograd_in_the_projection_layout_matches_contiguous_bit_for_bit():
+    """Q, K, V as [B,H,N,128] views of [B,N,H,128] tensors (no copies): the
+    forward output and the three gradients equal the contiguous run's bits."""
+    w = synth.custom("bwd_bnhd", 1, 3, 500, seed=95, k_offset_std=2.0, n_outliers=2, outlier_factor=20.0)
+    d = synth.generate(w)
+    dO = _dout((1, 3, 500, 128), seed=15).cuda()
+    runs = []
+    for layout in ("bhnd", "bnhd"):
+        if layout == "bhnd":
+            leaves = [d[t].cuda().requires_grad_(True) for t in "qkv"]
+            views = leaves
+        else:
+            leaves = [d[t].transpose(1, 2).contiguous().cuda().requires_grad_(True) for t in "qkv"]
+            views = [x.transpose(1, 2) for x in leaves]
+        o = fa().fp4_attention(*views)
+        o.backward(dO)
+        grads = [x.grad if layout == "bhnd" else x.grad.transpose(1, 2) for x in leaves]
+        runs.append([o.detach()] + grads)
+    for a, b in zip(*runs):
+        assert torch.equal(a.contiguous(), b.contiguous())
+    assert runs[1][0].stride() == runs[1][0].transpose(1, 2).contiguous().transpose(1, 2).stride()
