@@ -5,7 +5,7 @@
 // queries and keys are quantised for an NVFP4 attention kernel; P and V stay
 // in BF16.  This kernel is written for sm_100a:
 //   * one CTA per (head, 256 queries) = two 128-row query tiles that share
-//     every K/V tile loaded into shared memory; 320 threads:
+//     every K/V tile loaded into shared memory; 384 threads:
 //       warps 0-3  softmax of query tile 0, warps 4-7 softmax of tile 1 (one
 //                  warp per TMEM sub-partition, one query row per thread);
 //       warp 8     producer: scale-factor atoms (plain loads) and TMA copies
@@ -15,6 +15,8 @@
 //                  (tcgen05.cp), S_i = Q_i K^T with tcgen05.mma
 //                  kind::mxf4nvf4 (block16 UE4M3 scales) into TMEM, and
 //                  O_i += P_i V with tcgen05.mma kind::f16 from shared memory;
+//       warps 10-11 idle: they complete the third warpgroup, whose registers
+//                  go to the softmax warpgroups (setmaxnreg 216 / 64);
 //   * P_i goes to shared memory (K-major, 32-byte swizzle, one 4 KB panel per
 //     16 keys), not back into TMEM, so S_i is free as soon as its softmax
 //     warps have loaded it: S_i of the next stage is computed while they
