@@ -267,19 +267,21 @@ __global__ void __launch_bounds__(PRO_THREADS, 2) prologue_kernel(const __grid_c
             for (int rr = 0; rr < 16; ++rr) kw[rr] = *reinterpret_cast<const uint2*>(hb + swz(16 * warp + rr, j) + in_chunk);
             __syncthreads();
             release(buf);
+            // |k| is checked once per thread against 2^20 (out-of-range keys make
+            // the outputs unspecified and raise the status; non-finite keys are
+            // also caught by the K tiles' transform of the same rows)
             long long acc[4] = {0, 0, 0, 0};
-            bool bad = false;
+            float kmax = 0.0f;
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
                 const float v[4] = {bf16lo(kw[rr].x), bf16hi(kw[rr].x), bf16lo(kw[rr].y), bf16hi(kw[rr].y)};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const bool in_range = fabsf(v[c]) < kKeyLimit;
-                    acc[c] += in_range ? __float2ll_rn(__fmul_rn(v[c], kTwo24)) : 0ll;
-                    bad |= !in_range;
+                    acc[c] += __float2ll_rn(__fmul_rn(v[c], kTwo24));
+                    kmax = fmaxf(kmax, fabsf(v[c]));
                 }
             }
-            if (bad) set_status(a.status, FP4ATTN_ERR_RANGE);
+            if (!(kmax < kKeyLimit)) set_status(a.status, FP4ATTN_ERR_RANGE);
 #pragma unroll
             for (int c = 0; c < 4; ++c) sm.kpart[warp][4 * lane + c] = acc[c];
             __syncthreads();
