@@ -306,6 +306,13 @@ int fp4attn_probe_qk_tile(const uint8_t* q_codes_dev, const uint8_t* q_scales_de
 int fp4attn_probe_pv_tile(const void* p_bf16_dev, const void* v_bf16_dev, float* o_out_dev,
                           cudaStream_t stream);
 
+/* Testing: the block-scale quotient amax / 6 is computed without a divide
+ * (one multiply by fl(1/6) and an FMA refinement).  This checks it against the
+ * IEEE quotient for every non-negative finite fp32 value (synchronous).
+ *   result_dev : device uint32[2] out: [0] the number of mismatches, [1] the
+ *     smallest mismatching bit pattern (0xFFFFFFFF if none). */
+int fp4attn_probe_div6(uint32_t* result_dev, cudaStream_t stream);
+
 /* Runs the bounded mbarrier wait of the attention kernel on a barrier that
  * nothing arrives at, with the given limit; the kernel must give up and write
  * FP4ATTN_ERR_TIMEOUT into *status_dev (device int32, set to 0 first). */

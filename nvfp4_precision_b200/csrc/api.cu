@@ -393,6 +393,15 @@ int fp4attn_probe_pv_tile(const void* p, const void* v, float* o_out, cudaStream
     return st;
 }
 
+int fp4attn_probe_div6(uint32_t* result, cudaStream_t stream) {
+    if (!result || ((uintptr_t)result & 3)) return FP4ATTN_ERR_INVALID_ARG;
+    uint32_t init[2] = {0u, 0xFFFFFFFFu};
+    cudaError_t e = cudaMemcpyAsync(result, init, sizeof init, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = launch_div6_check(result, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    return launch_status(e);
+}
+
 int fp4attn_probe_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t stream) {
     if (!status || limit_ns > 10000000000ull) return FP4ATTN_ERR_INVALID_ARG;
     return launch_probe_wait_timeout(status, limit_ns, stream);

@@ -56,7 +56,27 @@ __global__ void encode_kernel(const float* __restrict__ x, int64_t n, uint8_t* e
     }
 }
 
+// Every non-negative finite fp32 bit pattern: div6_rn against the IEEE quotient.
+// res[0] counts mismatches, res[1] holds the smallest mismatching pattern.
+__global__ void div6_check_kernel(unsigned* res) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    unsigned count = 0;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < 0x7F800000u; i += stride) {
+        const float a = __uint_as_float(i);
+        if (__float_as_uint(div6_rn(a)) != __float_as_uint(__fdiv_rn(a, 6.0f))) {
+            ++count;
+            atomicMin(res + 1, i);
+        }
+    }
+    if (count) atomicAdd(res, count);
+}
+
 }  // namespace
+
+cudaError_t launch_div6_check(unsigned* res, cudaStream_t stream) {
+    div6_check_kernel<<<148 * 8, 256, 0, stream>>>(res);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
                            float* out, cudaStream_t stream) {

@@ -139,7 +139,7 @@ __device__ __forceinline__ float amax16(const float2* p, bool hi) {
 // Scale byte and 1/(g*scale) of one block with amax a.
 __device__ __forceinline__ void block_scale(float a, float g, bool g_is_one, const float* inv_tab, uint32_t& s,
                                             float& inv) {
-    float t = __fdiv_rn(a, 6.0f);
+    float t = div6_rn(a);
     if (!g_is_one) t = __fdiv_rn(t, g);
     s = cvt_e4m3(t);  // t >= +0: the E4M3 byte is the UE4M3 byte
     if (g_is_one) {

@@ -33,7 +33,7 @@ EXPORTS = (
     "fp4attn_dequant", "fp4attn_dequant_bf16", "fp4attn_backward", "fp4attn_backward_ex",
     "fp4attn_backward_workspace_bytes",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
-    "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout",
+    "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout", "fp4attn_probe_div6",
 )
 
 
@@ -101,6 +101,8 @@ def _load():
     L.fp4attn_probe_qk_tile.argtypes = [P, P, P, P, P, P]
     L.fp4attn_probe_pv_tile.restype = ctypes.c_int
     L.fp4attn_probe_pv_tile.argtypes = [P, P, P, P]
+    L.fp4attn_probe_div6.restype = ctypes.c_int
+    L.fp4attn_probe_div6.argtypes = [P, P]
     L.fp4attn_probe_wait_timeout.restype = ctypes.c_int
     L.fp4attn_probe_wait_timeout.argtypes = [P, U64, P]
     return L
@@ -393,6 +395,15 @@ def fp4attn_probe_pv_tile(p: torch.Tensor, v: torch.Tensor, stream=None) -> torc
     o = torch.empty((128, 128), dtype=torch.float32, device=p.device)
     _check(lib.fp4attn_probe_pv_tile(_ptr(p), _ptr(v), _ptr(o), _stream(stream)), "fp4attn_probe_pv_tile")
     return o
+
+
+def fp4attn_probe_div6(stream=None):
+    """(number of mismatches, smallest mismatching bit pattern) of the device
+    amax / 6 against the IEEE quotient over every non-negative finite fp32."""
+    res = torch.zeros(2, dtype=torch.int32, device="cuda")
+    _check(lib.fp4attn_probe_div6(_ptr(res), _stream(stream)), "fp4attn_probe_div6")
+    r = res.cpu().numpy().view("uint32")
+    return int(r[0]), int(r[1])
 
 
 def fp4attn_probe_wait_timeout(limit_ns: int, stream=None) -> int:

@@ -28,6 +28,13 @@ def _fp32_range(lo_exp, hi_exp, step=1):
     return np.arange(lo, hi, step, dtype=np.uint32).view(np.float32)
 
 
+def test_block_scale_quotient_is_the_ieee_quotient_for_every_input():
+    """The prologue computes amax / 6 with a multiply and an FMA refinement;
+    every non-negative finite fp32 amax gives the IEEE quotient's bits."""
+    count, first = fa().fp4attn_probe_div6()
+    assert count == 0, f"{count} mismatches, first at bits {first:#010x}"
+
+
 def test_device_codecs_match_oracle_over_dense_fp32_sweep():
     # every fp32 value with magnitude in [2^-12, 2^10) (both signs), plus zeros,
     # tiny, huge and infinite values
