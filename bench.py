@@ -402,24 +402,23 @@ def run_ours(args, rank, world, local):
         del qt, kt, vt, ot
 
     # ---- training-time backward (straight-through), outside the timed step:
-    # dequantised Q^, K^ of this step's codes, the step's O and lse, a random dO ----
+    # this step's NVFP4 codes, O and lse, a random dO ----
     training = None
     if not args.no_train:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         fa.fp4attn_quantize_qk(q, k, flags=0, out=out, workspace=ws, stream=stream)
         fa.fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, o=o, lse=lse,
                            workspace=ws, stream=stream)
-        qh = fa.fp4attn_dequant_bf16(out["q_codes"], out["q_scales"], stream=stream)
-        kh = fa.fp4attn_dequant_bf16(out["k_codes"], out["k_scales"], stream=stream)
+        cq = (out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"])
         g = torch.Generator(device=dev).manual_seed(17)
         dout = torch.randn((B, H, N, 128), generator=g, device=dev).to(torch.bfloat16)
         bws = torch.empty(fa.fp4attn_backward_workspace_bytes(B, H, N), dtype=torch.uint8, device=dev)
-        fa.fp4attn_backward(qh, kh, v, o, dout, lse, workspace=bws, stream=stream)
+        fa.fp4attn_backward(*cq, v, o, dout, lse, workspace=bws, stream=stream)
         reps = 2
         tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
         for e in tev:
             e[0].record(stream)
-            fa.fp4attn_backward(qh, kh, v, o, dout, lse, workspace=bws, stream=stream)
+            fa.fp4attn_backward(*cq, v, o, dout, lse, workspace=bws, stream=stream)
             e[1].record(stream)
         torch.cuda.synchronize(dev)
         st = fa.fp4attn_read_status(bws)
@@ -429,8 +428,8 @@ def run_ours(args, rank, world, local):
         f_bw = 2.5 * F  # five N x N x d products against the forward's two
         training = {"backward_ms": ms_bw, "backward_tflops": f_bw / (ms_bw * 1e-3) / 1e12,
                     "frac_bf16_sustained": f_bw / (ms_bw * 1e-3) / 1e12 / peaks["bf16_sustained"],
-                    "launches": 5}
-        del qh, kh, dout, bws
+                    "launches": 6}
+        del dout, bws
 
     csrc = os.path.join(ROOT, "nvfp4_precision_b200", "csrc")
     traffic = ATTN_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "attention.cu")), args.workload))

@@ -215,23 +215,24 @@ int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, 
  * "NVFP4 QAD": the 4-bit student trains with 4-bit math on from the first
  * step; the summary list: the training-time FP4 attention matches the
  * inference kernel).  The forward is the inference path (fp4attn_quantize_qk,
- * fp4attn_forward with lse) plus fp4attn_dequant_bf16 of the codes; the
- * backward below is a straight-through estimator: attention gradients at the
- * dequantised Q^ and K^, passed unchanged through the quantiser, then the
- * exact transforms differentiated:
+ * fp4attn_forward with lse); the backward below is a straight-through
+ * estimator: attention gradients at the dequantised Q^ = gQ Q~ and
+ * K^ = gK K~ (Q~, K~ the unit-scale values of the NVFP4 codes), passed
+ * unchanged through the quantiser, then the exact transforms differentiated:
  *   P = exp(scale Q^K^T - lse), dP = dO V^T, D = rowsum(dO * O),
  *   dS = P * (dP - D), dV = P^T dO, dQ^ = scale dS K^, dK^ = scale dS^T Q^,
  *   dq = c H dQ^, dk = c H (dK^ - mean_n dK^)   (c = 1/sqrt(128)).
- * P and dS are rounded to bf16 for the BF16 tensor-core products, which
- * accumulate in fp32; dq, dk, dv are bf16.
- *   qhat_dev, khat_dev : [B,H,N,128] bf16 unit-scale dequantised Q and K
- *     (block scale x E2M1, exact in bf16): fp4attn_dequant_bf16 with a NULL
- *     scale.
+ * The query-side kernel computes S from the codes with the forward's
+ * block-scaled FP4 MMA (the scores the forward's lse was taken over); the
+ * key-side kernel uses Q~, K~ in bf16 (exact), which this call dequantises
+ * into the workspace.  P and dS are rounded to bf16 for the BF16 tensor-core
+ * products, which accumulate in fp32; dq, dk, dv are bf16.  The global
+ * scales are applied as scalars (in the softmax scale and the dQ^ / dK^
+ * factors), never by rounding gQ * Q~ to bf16.
+ *   q_codes_dev, q_scales_dev, k_codes_dev, k_scales_dev : the forward's
+ *     NVFP4 Q and K from fp4attn_quantize_qk ([B,H,N,64] / [B,H,N,8]).
  *   q_gscale_dev, k_gscale_dev : the forward's global scales (device fp32
- *     scalars, finite and > 0), or NULL for 1.0.  Q^ = gQ * qhat and
- *     K^ = gK * khat; the scales are applied as scalars (in the softmax scale
- *     and the dQ^ / dK^ factors), never by rounding gQ * qhat to bf16, so the
- *     backward's scores equal the forward's.
+ *     scalars, finite and > 0), or NULL for 1.0.
  *   v_dev, o_dev, do_dev : [B,H,N,128] bf16: V, the forward's O and dL/dO.
  *   lse_dev : [B,H,N] fp32 from the forward.
  *   softmax_scale : that of the forward (<= 0 selects 1/sqrt(128)).
@@ -239,27 +240,28 @@ int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, 
  *   dq_dev, dk_dev, dv_dev : [B,H,N,128] bf16 out: gradients of the bf16 Q,
  *     K (the prologue's inputs) and V.
  *   workspace_dev : fp4attn_backward_workspace_bytes(s) bytes (status word
- *     first, so fp4attn_read_status works on it; about 512 bytes per row).
+ *     first, so fp4attn_read_status works on it; about 1 KB per row).
  * All tensors contiguous.  Device errors: FP4ATTN_ERR_RANGE for a bad global
- * scale; FP4ATTN_ERR_TIMEOUT if an internal
- * wait ran out. */
+ * scale; FP4ATTN_ERR_TIMEOUT if an internal wait ran out. */
 size_t fp4attn_backward_workspace_bytes(fp4attn_shape s);
-int fp4attn_backward(const void* qhat_dev, const void* khat_dev, const float* q_gscale_dev,
-                     const float* k_gscale_dev, const void* v_dev, const void* o_dev, const void* do_dev,
-                     const float* lse_dev, fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq_dev,
-                     void* dk_dev, void* dv_dev, void* workspace_dev, size_t workspace_bytes,
-                     cudaStream_t stream);
+int fp4attn_backward(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const uint8_t* k_codes_dev,
+                     const uint8_t* k_scales_dev, const float* q_gscale_dev, const float* k_gscale_dev,
+                     const void* v_dev, const void* o_dev, const void* do_dev, const float* lse_dev,
+                     fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq_dev, void* dk_dev,
+                     void* dv_dev, void* workspace_dev, size_t workspace_bytes, cudaStream_t stream);
 
 /* fp4attn_backward with V, O, dO and the outputs dq, dk, dv in one layout of
  * any element strides (fp4attn_strides; e.g. [B,N,H,128] as a QKV projection
- * writes them); qhat, khat and lse stay contiguous (the library's own
- * outputs).  The outputs' rows must not overlap one another or any input.
- * Errors as for fp4attn_backward; FP4ATTN_ERR_INVALID_ARG for a bad stride. */
-int fp4attn_backward_ex(const void* qhat_dev, const void* khat_dev, const float* q_gscale_dev,
-                        const float* k_gscale_dev, const void* v_dev, const void* o_dev, const void* do_dev,
-                        fp4attn_strides io_strides, const float* lse_dev, fp4attn_shape s, float softmax_scale,
-                        uint32_t flags, void* dq_dev, void* dk_dev, void* dv_dev, void* workspace_dev,
-                        size_t workspace_bytes, cudaStream_t stream);
+ * writes them); the codes, scales and lse keep their layouts (the library's
+ * own outputs).  The outputs' rows must not overlap one another or any
+ * input.  Errors as for fp4attn_backward; FP4ATTN_ERR_INVALID_ARG for a bad
+ * stride. */
+int fp4attn_backward_ex(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const uint8_t* k_codes_dev,
+                        const uint8_t* k_scales_dev, const float* q_gscale_dev, const float* k_gscale_dev,
+                        const void* v_dev, const void* o_dev, const void* do_dev, fp4attn_strides io_strides,
+                        const float* lse_dev, fp4attn_shape s, float softmax_scale, uint32_t flags,
+                        void* dq_dev, void* dk_dev, void* dv_dev, void* workspace_dev, size_t workspace_bytes,
+                        cudaStream_t stream);
 
 /* Decode NVFP4 rows to bf16: out = bf16(fl(fl(g * s) * e2m1)), exact when
  * g = 1.  codes_dev [rows,64], scales_dev [rows,8], gscale_dev scalar or

@@ -260,10 +260,11 @@ size_t fp4attn_backward_workspace_bytes(fp4attn_shape s) {
     return bws_bytes(bh, s.N > 0 ? s.N : 0);
 }
 
-int fp4attn_backward_ex(const void* qhat, const void* khat, const float* gq, const float* gk, const void* v,
-                        const void* o, const void* dout, fp4attn_strides io_strides, const float* lse,
-                        fp4attn_shape s, float softmax_scale, uint32_t flags, void* dq, void* dk, void* dv,
-                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int fp4attn_backward_ex(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                        const uint8_t* k_scales, const float* gq, const float* gk, const void* v, const void* o,
+                        const void* dout, fp4attn_strides io_strides, const float* lse, fp4attn_shape s,
+                        float softmax_scale, uint32_t flags, void* dq, void* dk, void* dv, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
     int st = check_shape(s);
     if (st != FP4ATTN_OK) return st;
     if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD)) return FP4ATTN_ERR_INVALID_ARG;
@@ -271,7 +272,7 @@ int fp4attn_backward_ex(const void* qhat, const void* khat, const float* gq, con
         return FP4ATTN_ERR_WORKSPACE;
     if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f) return FP4ATTN_ERR_INVALID_ARG;
     if (!empty(s)) {
-        const void* ptrs[] = {qhat, khat, v, o, dout, lse, dq, dk, dv};
+        const void* ptrs[] = {q_codes, q_scales, k_codes, k_scales, v, o, dout, lse, dq, dk, dv};
         for (const void* p : ptrs)
             if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
     }
@@ -284,8 +285,12 @@ int fp4attn_backward_ex(const void* qhat, const void* khat, const float* gq, con
     if (e != cudaSuccess) return launch_status(e);
     if (empty(s)) return FP4ATTN_OK;
     BwdArgs a;
-    a.qhat = static_cast<const __nv_bfloat16*>(qhat);
-    a.khat = static_cast<const __nv_bfloat16*>(khat);
+    a.q_codes = q_codes;
+    a.q_scales = q_scales;
+    a.k_codes = k_codes;
+    a.k_scales = k_scales;
+    a.qhat = reinterpret_cast<__nv_bfloat16*>(ws + bws_qt_offset(BH, s.N));
+    a.khat = reinterpret_cast<__nv_bfloat16*>(ws + bws_kt_offset(BH, s.N));
     a.gq = gq;
     a.gk = gk;
     a.v = static_cast<const __nv_bfloat16*>(v);
@@ -311,12 +316,12 @@ int fp4attn_backward_ex(const void* qhat, const void* khat, const float* gq, con
     return st;
 }
 
-int fp4attn_backward(const void* qhat, const void* khat, const float* gq, const float* gk, const void* v,
-                     const void* o, const void* dout, const float* lse, fp4attn_shape s, float softmax_scale,
-                     uint32_t flags, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                     cudaStream_t stream) {
-    return fp4attn_backward_ex(qhat, khat, gq, gk, v, o, dout, contiguous(s), lse, s, softmax_scale, flags, dq, dk,
-                               dv, workspace, workspace_bytes, stream);
+int fp4attn_backward(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                     const uint8_t* k_scales, const float* gq, const float* gk, const void* v, const void* o,
+                     const void* dout, const float* lse, fp4attn_shape s, float softmax_scale, uint32_t flags,
+                     void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return fp4attn_backward_ex(q_codes, q_scales, k_codes, k_scales, gq, gk, v, o, dout, contiguous(s), lse, s,
+                               softmax_scale, flags, dq, dk, dv, workspace, workspace_bytes, stream);
 }
 
 int fp4attn_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s, void* out,

@@ -17,8 +17,11 @@
 // Three kernels, all on the fifth-generation tensor cores (BF16 operands,
 // fp32 accumulators in TMEM):
 //   bwd_q_kernel  one CTA per (head, 128 queries): D of its rows (written for
-//                 the next kernel), then per 64-key stage S = Q^K^T and
-//                 dP = dO V^T (M=128, N=64), dS in registers written as bf16
+//                 the next kernel), then per 64-key stage S = Q~K~^T from the
+//                 NVFP4 codes with the forward's block-scaled MMA (the same
+//                 scores the forward's lse was taken over, at a quarter of a
+//                 BF16 product's cost) and dP = dO V^T (M=128, N=64), dS in
+//                 registers written as bf16
 //                 over the first 32 columns of S, dQ^ += dS K^ with dS read
 //                 from TMEM; epilogue dq = c H (scale dQ^) in registers.
 //   bwd_kv_kernel one CTA per (head, 128 keys): per 64-query stage
@@ -36,6 +39,7 @@
 // that runs out raises FP4ATTN_ERR_TIMEOUT and the CTA winds down.
 #include <cuda_bf16.h>
 
+#include "fp4_operands.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -132,6 +136,8 @@ struct BwdParams {
     long long io_sb, io_sh, io_sn;
     float* dk_acc;      // [BH, N, 128] fp32: scale * dK^
     float* partial;     // [BH, key tiles * 4, 128] fp32: column sums of scale * dK^ per warp
+    const uint64_t* q_scales;  // [BH, N] NVFP4 scale rows (8 UE4M3 bytes each)
+    const uint64_t* k_scales;
     bool hadamard;
     int* status;
     uint64_t limit_ns;
@@ -139,11 +145,19 @@ struct BwdParams {
 
 // ------------------------------------------------------------- dQ kernel --
 
+constexpr uint32_t QC_BYTES = BR * 64;  // 128 rows of 128 E2M1 codes, 64B swizzle
+constexpr uint32_t KC_BYTES = BS * 64;  // 64 rows
+constexpr uint32_t TM_SFQ = 384, TM_SFK = 392;  // scale factors: Q [384,392), K slots [392,400), [400,408)
+constexpr uint32_t IDESC_S4 = idesc_mxf4(BR, BS);
+
 struct __align__(1024) QSmem {
-    uint8_t q[TILE_R];               // Q^ tile, K-major
     uint8_t dout[TILE_R];            // dO tile, K-major
-    uint8_t k[STAGES][TILE_S];       // K^ stage: K-major for S, MN-major for dQ^ += dS K^
+    uint8_t k[STAGES][TILE_S];       // K~ stage (bf16), MN-major for dQ^ += dS K^
     uint8_t v[STAGES][TILE_S];       // V stage, K-major for dP
+    uint8_t qc[QC_BYTES];            // Q codes
+    uint8_t kc[STAGES][KC_BYTES];    // K codes of the stage
+    uint8_t qs_atom[2][512];         // scale-factor atoms for tcgen05.cp
+    uint8_t ks_atom[STAGES][2][512];
     uint64_t bar_q_full;
     uint64_t bar_kv_full[STAGES];
     uint64_t bar_kv_empty[STAGES];
@@ -155,9 +169,9 @@ struct __align__(1024) QSmem {
 };
 
 __global__ void __launch_bounds__(THREADS, 1)
-    bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const BwdParams p) {
+    bwd_q_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     QSmem& sm = *reinterpret_cast<QSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
@@ -194,26 +208,42 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int hb = bh / p.H, hh = bh - hb * p.H;
 
     if (warp == WARP_PRODUCER) {
-        // Q^ and dO once, then K^ and V of BS keys per stage.  Rows past N are
-        // filled with zeros by the copy.
+        // Q codes (with their scale atoms) and dO once, then per stage the K
+        // codes and scale atoms and the bf16 K~ and V of BS keys.  Rows past N
+        // are filled with zeros by the copies (scales: zero bytes).
         const uint32_t qf = smem_u32(&sm.bar_q_full);
+        load_scale_atoms(p.q_scales + (size_t)bh * N + q0, N - q0, sm.qs_atom[0], sm.qs_atom[1], lane);
+        fence_proxy_async_smem();
+        __syncwarp();
         if (lane == 0) {
-            mbar_arrive_expect_tx(qf, 2 * TILE_R);
-            tma_load_4d(smem_u32(sm.q), &tm_q, 0, q0, hh, hb, qf);
-            tma_load_4d(smem_u32(sm.q) + PANEL_R, &tm_q, 64, q0, hh, hb, qf);
+            mbar_arrive_expect_tx(qf, QC_BYTES + 2 * PANEL_R);
+            tma_load_3d(smem_u32(sm.qc), &tm_qc, 0, q0, bh, qf);
             tma_load_4d(smem_u32(sm.dout), &tm_do, 0, q0, hh, hb, qf);
             tma_load_4d(smem_u32(sm.dout) + PANEL_R, &tm_do, 64, q0, hh, hb, qf);
         }
+        // K scale rows are fetched one stage ahead: their load latency overlaps
+        // the wait for a free buffer instead of delaying the stage's copies
+        const uint64_t* ks_head = p.k_scales + (size_t)bh * N;
+        uint64_t ksc[4];
+        fetch_scales(ks_head, N < BS ? N : BS, lane, ksc);
         int issued = 0;
         for (int j = 0; j < T; ++j) {
             const int st = j % STAGES;
             if (j >= STAGES &&
                 !warp_wait(smem_u32(&sm.bar_kv_empty[st]), ((j / STAGES) - 1) & 1, abort_flag, p.status, limit))
                 break;
+            const int k0 = j * BS;
+            store_scale_atoms(ksc, sm.ks_atom[st][0], sm.ks_atom[st][1], lane);
+            if (j + 1 < T) {
+                const int rest = N - k0 - BS;
+                fetch_scales(ks_head + k0 + BS, rest < BS ? rest : BS, lane, ksc);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
             if (lane == 0) {
                 const uint32_t full = smem_u32(&sm.bar_kv_full[st]);
-                const int k0 = j * BS;
-                mbar_arrive_expect_tx(full, 2 * TILE_S);
+                mbar_arrive_expect_tx(full, KC_BYTES + 2 * TILE_S);
+                tma_load_3d(smem_u32(sm.kc[st]), &tm_kc, 0, k0, bh, full);
                 tma_load_4d(smem_u32(sm.k[st]), &tm_k, 0, k0, hh, hb, full);
                 tma_load_4d(smem_u32(sm.k[st]) + PANEL_S, &tm_k, 64, k0, hh, hb, full);
                 tma_load_4d(smem_u32(sm.v[st]), &tm_v, 0, k0, hh, hb, full);
@@ -229,20 +259,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         const bool leader = elect_one_sync();
-        const uint64_t qd = kmajor_desc(sm.q);
+        const uint64_t qcd = codes_desc(sm.qc, 0);
+        const uint64_t kcd0 = codes_desc(sm.kc[0], 0);     // stage st: + st * KC_BYTES / 16
+        const uint64_t kad0 = atom_desc(sm.ks_atom[0][0]);  // stage st: + 64 st, half h: + 32 h
         const uint64_t dod = kmajor_desc(sm.dout);
-        const uint64_t kd0 = kmajor_desc(sm.k[0]);   // stage st: + st * TILE_S / 16
-        const uint64_t vd0 = kmajor_desc(sm.v[0]);
+        const uint64_t vd0 = kmajor_desc(sm.v[0]);          // stage st: + st * TILE_S / 16
         const uint64_t kmn0 = mn_desc(sm.k[0], PANEL_S);
-        constexpr uint64_t TD = TILE_S >> 4;
+        constexpr uint64_t TD = TILE_S >> 4, KCD = KC_BYTES >> 4, AD = (2 * 512) >> 4;
         auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, p.status, limit));
         };
-        auto scores = [&](int b, int st) {  // S_b = Q^ K^T, dP_b = dO V^T
-#pragma unroll
-            for (int ks = 0; ks < 128 / 16; ++ks)
-                mma_bf16_ss(tmem + TM_X + BS * b, qd + kstep(PANEL_R, ks), kd0 + TD * st + kstep(PANEL_S, ks),
-                            IDESC_ST, ks > 0 ? 1u : 0u);
+        // S_b = Q~ K~^T from the codes (K scale factors of stage j into slot
+        // j & 1: the stage two back, which used that slot, was issued before),
+        // dP_b = dO V^T
+        auto scores = [&](int b, int st, int j) {
+            const uint32_t sfk = TM_SFK + 8u * (uint32_t)(j & 1);
+            tmem_cp_32x128b_x4(tmem + sfk, kad0 + AD * st);
+            tmem_cp_32x128b_x4(tmem + sfk + 4, kad0 + AD * st + 32);
+            mma_mxf4nvf4(tmem + TM_X + BS * b, qcd, kcd0 + KCD * st, IDESC_S4, tmem + TM_SFQ, tmem + sfk, 0u);
+            mma_mxf4nvf4(tmem + TM_X + BS * b, qcd + 2, kcd0 + KCD * st + 2, IDESC_S4, tmem + TM_SFQ + 4,
+                         tmem + sfk + 4, 1u);
 #pragma unroll
             for (int ks = 0; ks < 128 / 16; ++ks)
                 mma_bf16_ss(tmem + TM_Y + BS * b, dod + kstep(PANEL_R, ks), vd0 + TD * st + kstep(PANEL_S, ks),
@@ -257,6 +293,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_commit(smem_u32(&sm.bar_kv_empty[st]));
         };
         bool ok = wait(smem_u32(&sm.bar_q_full), 0);
+        if (ok && leader) {
+            tc_fence_after();
+            const uint64_t qad = atom_desc(sm.qs_atom[0]);
+            tmem_cp_32x128b_x4(tmem + TM_SFQ, qad);
+            tmem_cp_32x128b_x4(tmem + TM_SFQ + 4, qad + 32);
+        }
+        __syncwarp();
         for (int j = 0; ok && j < T; ++j) {
             const int st = j % STAGES;
             if (!wait(smem_u32(&sm.bar_kv_full[st]), (j / STAGES) & 1)) {
@@ -265,7 +308,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             if (leader) {
                 tc_fence_after();
-                scores(j & 1, st);
+                scores(j & 1, st, j);
             }
             __syncwarp();
             if (j > 0) {
@@ -341,17 +384,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_ld32(tmem + lane_base + TM_Y + BS * b + 32, &dr[32]);
             tmem_wait_ld();
             const int nvalid = N - j * BS;  // keys of this stage that exist
+            const float2 c2 = make_float2(c, c), nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-Dr, -Dr);
             uint32_t pk[BS / 2];
 #pragma unroll
             for (int k = 0; k < BS / 2; ++k) {
-                float ds[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int kk = 2 * k + e;
-                    const float pr = ex2_approx(fmaf(__uint_as_float(sr[kk]), c, -lse2));
-                    ds[e] = (kk < nvalid) ? pr * (__uint_as_float(dr[kk]) - Dr) : 0.0f;
-                }
-                pk[k] = pack_bf16x2(ds[0], ds[1]);
+                // exponentials: 3 of every 8 pairs on the FMA-pipe polynomial, the
+                // rest on MUFU (as in the forward), packed fp32x2 arithmetic
+                const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
+                                            c2, nl2);
+                const float2 pr = ((k & 7) < 3) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                float2 ds = __fmul2_rn(pr, __fadd2_rn(make_float2(__uint_as_float(dr[2 * k]),
+                                                                  __uint_as_float(dr[2 * k + 1])), nd2));
+                if (2 * k >= nvalid) ds.x = 0.0f;
+                if (2 * k + 1 >= nvalid) ds.y = 0.0f;
+                pk[k] = pack_bf16x2(ds.x, ds.y);
             }
             tmem_st32(tmem + lane_base + TM_X + BS * b, pk);  // dS over the first 32 columns of S_b
             tmem_wait_st();
@@ -773,9 +819,15 @@ bool make_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, ui
 int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     const int B = a.BH / a.H;
-    CUtensorMap q_r, do_r, k_s, v_s, k_r, v_r, q_s, do_s;
+    // unit-scale Q~, K~ in bf16 (exact) for the dK / dV kernel and the dQ^ product
+    const int64_t rows = (int64_t)a.BH * a.N;
+    if (launch_dequant_bf16(a.q_codes, a.q_scales, nullptr, rows, a.qhat, stream) != cudaSuccess ||
+        launch_dequant_bf16(a.k_codes, a.k_scales, nullptr, rows, a.khat, stream) != cudaSuccess)
+        return FP4ATTN_ERR_CUDA;
+    CUtensorMap qc_r, kc_s, do_r, k_s, v_s, k_r, v_r, q_s, do_s;
     const Strides cs = contiguous_strides(a.H, a.N);  // Q~, K~: the library's own contiguous tensors
-    if (!make_map(&q_r, a.qhat, B, a.H, a.N, BR, cs) || !make_map(&do_r, a.dout, B, a.H, a.N, BR, a.io) ||
+    if (!make_code_map(&qc_r, a.q_codes, a.BH, a.N, BR) || !make_code_map(&kc_s, a.k_codes, a.BH, a.N, BS) ||
+        !make_map(&do_r, a.dout, B, a.H, a.N, BR, a.io) ||
         !make_map(&k_s, a.khat, B, a.H, a.N, BS, cs) || !make_map(&v_s, a.v, B, a.H, a.N, BS, a.io) ||
         !make_map(&k_r, a.khat, B, a.H, a.N, BR, cs) || !make_map(&v_r, a.v, B, a.H, a.N, BR, a.io) ||
         !make_map(&q_s, a.qhat, B, a.H, a.N, BS, cs) || !make_map(&do_s, a.dout, B, a.H, a.N, BS, a.io))
@@ -795,6 +847,8 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     p.scale_log2 = p.scale * kLog2e;
     p.gq = a.gq;
     p.gk = a.gk;
+    p.q_scales = reinterpret_cast<const uint64_t*>(a.q_scales);
+    p.k_scales = reinterpret_cast<const uint64_t*>(a.k_scales);
     p.lse = a.lse;
     p.dsum = a.dsum;
     p.o = a.o;
@@ -810,7 +864,7 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;
     const dim3 grid((a.N + BR - 1) / BR, a.BH);
-    bwd_q_kernel<<<grid, THREADS, smem_q, stream>>>(q_r, do_r, k_s, v_s, p);
+    bwd_q_kernel<<<grid, THREADS, smem_q, stream>>>(qc_r, do_r, kc_s, k_s, v_s, p);
     if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
     bwd_kv_kernel<<<grid, THREADS, smem_kv, stream>>>(k_r, v_r, q_s, do_s, p);
     if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
@@ -818,7 +872,6 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
         colsum_kernel<<<a.BH, 128, 0, stream>>>(a.partial, 4 * (int)grid.x, a.colsum);
         if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
     }
-    const int64_t rows = (int64_t)a.BH * a.N;
     const int64_t want = (rows + 7) / 8;  // 8 warps per block, one row each
     const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
     ste_k_kernel<<<blocks, 256, 0, stream>>>(a.dk_acc, a.colsum, a.N, a.H, rows, !(a.flags & FP4ATTN_NO_SMOOTH_K),

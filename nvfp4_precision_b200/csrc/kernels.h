@@ -102,7 +102,8 @@ struct FwdBf16Args {
 
 // Backward workspace: [0,256) status word and spare; then D [BH*N] fp32,
 // column sums [BH*128] fp32, per-warp column sums [BH*ceil(N/128)*4*128] fp32,
-// scale * dK^ [BH*N*128] fp32 (each 256-aligned).
+// scale * dK^ [BH*N*128] fp32, unit-scale Q~ and K~ [BH*N*128] bf16 each
+// (each 256-aligned).
 inline size_t bws_align(size_t b) { return (b + 255) / 256 * 256; }
 inline size_t bws_dsum_offset() { return WS_STATUS_BYTES; }
 inline size_t bws_colsum_offset(int64_t BH, int64_t N) { return bws_dsum_offset() + bws_align((size_t)(BH * N) * 4); }
@@ -112,11 +113,17 @@ inline size_t bws_partial_offset(int64_t BH, int64_t N) {
 inline size_t bws_dk_offset(int64_t BH, int64_t N) {
     return bws_partial_offset(BH, N) + bws_align((size_t)BH * ((N + 127) / 128) * 4 * D * 4);
 }
-inline size_t bws_bytes(int64_t BH, int64_t N) { return bws_dk_offset(BH, N) + bws_align((size_t)(BH * N) * D * 4); }
+inline size_t bws_qt_offset(int64_t BH, int64_t N) { return bws_dk_offset(BH, N) + bws_align((size_t)(BH * N) * D * 4); }
+inline size_t bws_kt_offset(int64_t BH, int64_t N) { return bws_qt_offset(BH, N) + bws_align((size_t)(BH * N) * D * 2); }
+inline size_t bws_bytes(int64_t BH, int64_t N) { return bws_kt_offset(BH, N) + bws_align((size_t)(BH * N) * D * 2); }
 
 struct BwdArgs {
-    const __nv_bfloat16* qhat;  // unit-scale dequantised Q and K, [B,H,N,128] contiguous
-    const __nv_bfloat16* khat;
+    const uint8_t* q_codes;     // the forward's NVFP4 Q and K ([B,H,N,64] codes, [B,H,N,8] scales)
+    const uint8_t* q_scales;
+    const uint8_t* k_codes;
+    const uint8_t* k_scales;
+    __nv_bfloat16* qhat;        // workspace: unit-scale dequantised Q and K, [B,H,N,128]
+    __nv_bfloat16* khat;
     const float* gq;            // global scales (device scalars) or nullptr for 1
     const float* gk;
     const __nv_bfloat16* v;

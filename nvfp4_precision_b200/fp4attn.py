@@ -82,11 +82,11 @@ def _load():
     L.fp4attn_backward_workspace_bytes.restype = ctypes.c_size_t
     L.fp4attn_backward_workspace_bytes.argtypes = [Shape]
     L.fp4attn_backward.restype = ctypes.c_int
-    L.fp4attn_backward.argtypes = [P, P, P, P, P, P, P, P, Shape, ctypes.c_float, U32, P, P, P, P, ctypes.c_size_t,
-                                   P]
+    L.fp4attn_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, Shape, ctypes.c_float, U32, P, P, P, P,
+                                   ctypes.c_size_t, P]
     L.fp4attn_backward_ex.restype = ctypes.c_int
-    L.fp4attn_backward_ex.argtypes = [P, P, P, P, P, P, P, Strides, P, Shape, ctypes.c_float, U32, P, P, P, P,
-                                      ctypes.c_size_t, P]
+    L.fp4attn_backward_ex.argtypes = [P, P, P, P, P, P, P, P, P, Strides, P, Shape, ctypes.c_float, U32, P, P, P,
+                                      P, ctypes.c_size_t, P]
     L.fp4attn_dequant.restype = ctypes.c_int
     L.fp4attn_dequant.argtypes = [P, P, P, Shape, P, P]
     L.fp4attn_read_status.restype = ctypes.c_int
@@ -290,18 +290,16 @@ def fp4attn_backward_workspace_bytes(B: int, H: int, N: int, D: int = 128) -> in
     return int(lib.fp4attn_backward_workspace_bytes(Shape(B, H, N, D)))
 
 
-def fp4attn_backward(qhat, khat, v, o, dout, lse, softmax_scale: float = 0.0, flags: int = 0,
-                     workspace: Optional[torch.Tensor] = None, stream=None, q_gscale: Optional[torch.Tensor] = None,
-                     k_gscale: Optional[torch.Tensor] = None):
+def fp4attn_backward(q_codes, q_scales, k_codes, k_scales, v, o, dout, lse, softmax_scale: float = 0.0,
+                     flags: int = 0, workspace: Optional[torch.Tensor] = None, stream=None,
+                     q_gscale: Optional[torch.Tensor] = None, k_gscale: Optional[torch.Tensor] = None):
     """Straight-through backward of the FP4 attention (see include/fp4attn.h):
-    bf16 [B,H,N,128] unit-scale dequantised Q~, K~ (fp4attn_dequant_bf16 with
-    no scale, contiguous), V, the forward's O, dL/dO (one layout of any
-    strides with contiguous channels, e.g. views of [B,N,H,128] tensors),
-    fp32 lse [B,H,N], and the forward's global scales (device scalars, None
-    for 1).  Returns (dq, dk, dv, workspace): bf16 gradients of the bf16 Q, K,
-    V inputs of the forward, in the layout of V."""
-    for t in (qhat, khat):
-        assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.shape == v.shape
+    the forward's NVFP4 Q and K (codes and scales from fp4attn_quantize_qk)
+    and global scales (device scalars, None for 1), V, the forward's O, dL/dO
+    (one layout of any strides with contiguous channels, e.g. views of
+    [B,N,H,128] tensors) and fp32 lse [B,H,N].  Returns (dq, dk, dv,
+    workspace): bf16 gradients of the bf16 Q, K, V inputs of the forward, in
+    the layout of V."""
     st = strides_of(v)
     for t in (o, dout):
         assert t.dtype == torch.bfloat16 and t.shape == v.shape and t.stride() == v.stride(), \
@@ -309,11 +307,12 @@ def fp4attn_backward(qhat, khat, v, o, dout, lse, softmax_scale: float = 0.0, fl
     assert v.dtype == torch.bfloat16
     assert lse.dtype == torch.float32 and lse.is_contiguous()
     B, H, N, D = v.shape
+    assert q_codes.shape == (B, H, N, 64) and k_codes.shape == (B, H, N, 64)
     if workspace is None:
         workspace = torch.empty(fp4attn_backward_workspace_bytes(B, H, N), dtype=torch.uint8, device=v.device)
     dq, dk, dv = (torch.empty_strided(v.shape, v.stride(), dtype=torch.bfloat16, device=v.device) for _ in range(3))
-    rc = lib.fp4attn_backward_ex(_ptr(qhat), _ptr(khat), _ptr(q_gscale), _ptr(k_gscale), _ptr(v), _ptr(o),
-                                 _ptr(dout), st, _ptr(lse), Shape(B, H, N, D),
+    rc = lib.fp4attn_backward_ex(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(q_gscale),
+                                 _ptr(k_gscale), _ptr(v), _ptr(o), _ptr(dout), st, _ptr(lse), Shape(B, H, N, D),
                                  float(softmax_scale), int(flags), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                                  workspace.numel(), _stream(stream))
     _check(rc, "fp4attn_backward_ex")
@@ -335,22 +334,21 @@ class FP4AttentionSTE(torch.autograd.Function):
         o = torch.empty_strided(v.shape, v.stride(), dtype=torch.bfloat16, device=v.device)
         o, lse = fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, gq, gk,
                                  softmax_scale=softmax_scale, o=o, want_lse=True, workspace=out["workspace"])
-        qhat = fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])  # unit scale: exact in bf16
-        khat = fp4attn_dequant_bf16(out["k_codes"], out["k_scales"])
+        codes = (out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"])
         st = fp4attn_read_status(out["workspace"])
         if st != OK:
             raise Fp4AttnError(st, "FP4AttentionSTE.forward (device)")
-        ctx.save_for_backward(qhat, khat, v, o, lse, gq, gk)
+        ctx.save_for_backward(*codes, v, o, lse, gq, gk)
         ctx.softmax_scale, ctx.flags = softmax_scale, flags
         return o
 
     @staticmethod
     def backward(ctx, do):
-        qhat, khat, v, o, lse, gq, gk = ctx.saved_tensors
+        qc, qs, kc, ks, v, o, lse, gq, gk = ctx.saved_tensors
         do = do.to(torch.bfloat16)
         if do.stride() != v.stride():
             do = torch.empty_strided(v.shape, v.stride(), dtype=torch.bfloat16, device=v.device).copy_(do)
-        dq, dk, dv, ws = fp4attn_backward(qhat, khat, v, o, do, lse, ctx.softmax_scale, ctx.flags,
+        dq, dk, dv, ws = fp4attn_backward(qc, qs, kc, ks, v, o, do, lse, ctx.softmax_scale, ctx.flags,
                                           q_gscale=gq, k_gscale=gk)
         st = fp4attn_read_status(ws)
         if st != OK:

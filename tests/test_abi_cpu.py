@@ -119,15 +119,18 @@ def test_backward_validation_before_launch(fa):
     f = fa.lib.fp4attn_backward
     shape = S(1, 2, 128, 128)
     wsb = fa.fp4attn_backward_workspace_bytes(1, 2, 128)
-    assert wsb >= 256 + 2 * 128 * 4 + 2 * 128 * 4 + 2 * 128 * 128 * 4
-    assert f(p, p, None, None, p, p, p, p, S(1, 2, 128, 64), 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_UNSUPPORTED
-    assert f(p, p, None, None, p, p, p, p, shape, 0.0, 0, p, p, p, p, wsb - 16, None) == fa.ERR_WORKSPACE
-    assert f(p, p, None, None, p, p, p, p, shape, 0.0, 8, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
-    assert f(p, p, None, None, p, p, p, p, shape, float("nan"), 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
-    assert f(p, p, None, None, p, p, p, None, shape, 0.0, 0, p, p, p, p, wsb, None) == fa.ERR_INVALID_ARG
-    assert f(p, p, None, None, p, p, p, p, shape, 0.0, 0, p, ctypes.c_void_p(4104), p, p, wsb, None) \
-        == fa.ERR_INVALID_ARG
-    assert f(p, p, ctypes.c_void_p(4098), None, p, p, p, p, shape, 0.0, 0, p, p, p, p, wsb, None) \
-        == fa.ERR_INVALID_ARG
+    assert wsb >= 256 + 2 * 128 * 4 + 2 * 128 * 4 + 2 * 128 * 128 * 4 + 2 * 2 * 128 * 128 * 2
+
+    def b(codes=p, g=None, lse=p, dk=p, flags=0, scale=0.0, sh=shape, ws=wsb):
+        return f(codes, p, p, p, g, None, p, p, p, lse, sh, scale, flags, p, dk, p, p, ws, None)
+
+    assert b(sh=S(1, 2, 128, 64)) == fa.ERR_UNSUPPORTED
+    assert b(ws=wsb - 16) == fa.ERR_WORKSPACE
+    assert b(flags=8) == fa.ERR_INVALID_ARG
+    assert b(scale=float("nan")) == fa.ERR_INVALID_ARG
+    assert b(lse=None) == fa.ERR_INVALID_ARG
+    assert b(codes=None) == fa.ERR_INVALID_ARG
+    assert b(dk=ctypes.c_void_p(4104)) == fa.ERR_INVALID_ARG
+    assert b(g=ctypes.c_void_p(4098)) == fa.ERR_INVALID_ARG
     d = fa.lib.fp4attn_dequant_bf16
     assert d(p, ctypes.c_void_p(4100), None, shape, p, None) == fa.ERR_INVALID_ARG

@@ -50,9 +50,8 @@ def _gpu_step(d, dO, flags=0, scale=0.0):
     o, lse = fa().fp4attn_forward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v,
                                   softmax_scale=scale, want_lse=True, workspace=out["workspace"])
     assert fa().fp4attn_read_status(out["workspace"]) == 0
-    qh = fa().fp4attn_dequant_bf16(out["q_codes"], out["q_scales"])
-    kh = fa().fp4attn_dequant_bf16(out["k_codes"], out["k_scales"])
-    dq, dk, dv, ws = fa().fp4attn_backward(qh, kh, v, o, dO.cuda(), lse, scale, flags)
+    dq, dk, dv, ws = fa().fp4attn_backward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"], v, o,
+                                           dO.cuda(), lse, scale, flags)
     assert fa().fp4attn_read_status(ws) == 0
     return dq.float().cpu().numpy(), dk.float().cpu().numpy(), dv.float().cpu().numpy()
 
@@ -71,8 +70,8 @@ def _bf16(x):
 
 
 def _kernel_parity(d, dO, flags=0, scale=None):
-    """Same inputs on both sides: the oracle's codes, dequantised Q^ and K^,
-    O (rounded to bf16) and lse."""
+    """Same inputs on both sides: the oracle's codes, its O (rounded to bf16)
+    and lse."""
     B, H, N, _ = d["q"].shape
     vb = synth.bf16_bits(d["v"])
     codes = oracle.quantize_qk(synth.bf16_bits(d["q"]), synth.bf16_bits(d["k"]), flags=flags)
@@ -84,8 +83,9 @@ def _kernel_parity(d, dO, flags=0, scale=None):
         for h in range(H):
             O[b, h], L[b, h] = oracle.attention_head(qh[b, h], kh[b, h], vb[b, h], scale)
     o_bf = _bf16(O)
-    dq, dk, dv, ws = fa().fp4attn_backward(_bf16(qh).cuda(), _bf16(kh).cuda(), d["v"].cuda(), o_bf.cuda(),
-                                           dO.cuda(), torch.from_numpy(L.astype(np.float32)).cuda(),
+    t = lambda key: torch.from_numpy(np.ascontiguousarray(codes[key])).cuda()
+    dq, dk, dv, ws = fa().fp4attn_backward(t("q_codes"), t("q_scales"), t("k_codes"), t("k_scales"), d["v"].cuda(),
+                                           o_bf.cuda(), dO.cuda(), torch.from_numpy(L.astype(np.float32)).cuda(),
                                            0.0 if scale is None else scale, flags)
     assert fa().fp4attn_read_status(ws) == 0
     ref = oracle.attention_backward(codes["q_codes"], codes["q_scales"], codes["k_codes"], codes["k_scales"], vb,
@@ -212,9 +212,9 @@ def test_fake_quant_forward_matches_the_fp4_kernel_within_1pct_of_quantisation_e
 def test_autograd_with_dynamic_scales_and_flags():
     """fp4_attention with the dynamic per-tensor scales and each transform off:
     gradients against the oracle's (same g, end-to-end bounds).  The backward
-    gets the unit-scale Q~, K~ (exact in bf16) and g as scalars: rounding
-    g * Q~ to bf16 instead would move the scores of these outlier-heavy keys
-    (lse up to about 360) by tenths of a unit and the gradients by over 10%."""
+    works on the unit-scale Q~, K~ and takes g as scalars: rounding g * Q~ to
+    bf16 instead would move the scores of these outlier-heavy keys (lse up to
+    about 360) by tenths of a unit and the gradients by over 10%."""
     w = synth.custom("bwd_dyn", 1, 2, 400, seed=91, k_offset_std=2.0, n_outliers=2, outlier_factor=20.0)
     d = synth.generate(w)
     dO = _dout((1, 2, 400, 128), seed=11)
@@ -233,9 +233,9 @@ def test_autograd_with_dynamic_scales_and_flags():
 
 
 def test_backward_kernel_parity_with_global_scales():
-    """Static global scales gQ = 0.37, gK = 1.9: the backward gets the unit-scale
-    Q~, K~ (exact in bf16) and the scales as scalars; same inputs on both sides
-    (the oracle's O rounded to bf16 and its lse), tight bounds."""
+    """Static global scales gQ = 0.37, gK = 1.9 (the scales enter the backward
+    as scalars); same inputs on both sides (the oracle's codes, its O rounded
+    to bf16 and its lse), tight bounds."""
     gq, gk = 0.37, 1.9
     w = synth.custom("bwd_g", 1, 2, 333, seed=93, k_offset_std=2.0, n_outliers=2, outlier_factor=20.0)
     d = synth.generate(w)
@@ -249,12 +249,11 @@ def test_backward_kernel_parity_with_global_scales():
                                                  oracle.dequant(codes["k_codes"][0, h], codes["k_scales"][0, h], gk),
                                                  vb[0, h])
     o_bf = _bf16(O)
-    qt = _bf16(oracle.dequant(codes["q_codes"], codes["q_scales"])).cuda()
-    kt = _bf16(oracle.dequant(codes["k_codes"], codes["k_scales"])).cuda()
+    t = lambda key: torch.from_numpy(np.ascontiguousarray(codes[key])).cuda()
     g = lambda x: torch.tensor([x], dtype=torch.float32, device="cuda")
-    dq, dk, dv, ws = fa().fp4attn_backward(qt, kt, d["v"].cuda(), o_bf.cuda(), dO.cuda(),
-                                           torch.from_numpy(L.astype(np.float32)).cuda(), q_gscale=g(gq),
-                                           k_gscale=g(gk))
+    dq, dk, dv, ws = fa().fp4attn_backward(t("q_codes"), t("q_scales"), t("k_codes"), t("k_scales"), d["v"].cuda(),
+                                           o_bf.cuda(), dO.cuda(), torch.from_numpy(L.astype(np.float32)).cuda(),
+                                           q_gscale=g(gq), k_gscale=g(gk))
     assert fa().fp4attn_read_status(ws) == 0
     rq, rk, rv = oracle.attention_backward(codes["q_codes"], codes["q_scales"], codes["k_codes"], codes["k_scales"],
                                            vb, dO.double().numpy(), gq, gk, O=o_bf.double().numpy())

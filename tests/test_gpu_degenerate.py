@@ -79,6 +79,7 @@ def test_empty_shapes_through_the_general_entry_points():
         assert ob.shape == (B, H, N, 128)
         z = torch.zeros((B, H, N, 128), dtype=torch.bfloat16, device=dev)
         lse = torch.zeros((B, H, N), dtype=torch.float32, device=dev)
-        dq, dk, dv, ws = fa().fp4attn_backward(z, z, z, z, z, lse)
+        dq, dk, dv, ws = fa().fp4attn_backward(out["q_codes"], out["q_scales"], out["k_codes"], out["k_scales"],
+                                               z, z, z, lse)
         assert fa().fp4attn_read_status(ws) == 0 and dq.shape == z.shape
         assert fa().fp4attn_dequant_bf16(out["q_codes"], out["q_scales"]).shape == (B, H, N, 128)
