@@ -44,7 +44,7 @@ PROLOGUE_BYTES_PER_ELEMENT = 5.125  # Q,K bf16 read (2+2) + codes (0.5+0.5) + sc
 # kernel source they were measured on and the workload; a changed kernel reports
 # null until it is profiled again (profiles/ holds the commands).
 ATTN_TRAFFIC_BYTES = {
-    ("287f509948c38120", "clip15s"): 2.416e9 + 1.372e9,
+    ("2e4a3044e0d72f66", "clip15s"): 2.416e9 + 1.372e9,
 }
 PROLOGUE_TRAFFIC_BYTES = {
     ("2cfa9c01d2643c07", "clip15s"): 2.703e9 + 0.725e9,
