@@ -47,7 +47,7 @@ ATTN_TRAFFIC_BYTES = {
     ("2e4a3044e0d72f66", "clip15s"): 2.416e9 + 1.372e9,
 }
 PROLOGUE_TRAFFIC_BYTES = {
-    ("2cfa9c01d2643c07", "clip15s"): 2.703e9 + 0.725e9,
+    ("2abaa5cb75d16bd1", "clip15s"): 2.703e9 + 0.723e9,
 }
 
 
