@@ -14,8 +14,8 @@
 //   dQ^ = scale dS K^,  dK^ = scale dS^T Q^,  dV = P^T dO,
 //   dq = c H dQ^,  dk = c H (dK^ - mean_n dK^)   (c = 1/sqrt(128)).
 //
-// Three kernels, all on the fifth-generation tensor cores (BF16 operands,
-// fp32 accumulators in TMEM):
+// Four kernels, the first two on the fifth-generation tensor cores (FP4
+// scores, BF16 products, fp32 accumulators in TMEM):
 //   bwd_q_kernel  one CTA per (head, 128 queries): D of its rows (written for
 //                 the next kernel), then per 64-key stage S = Q~K~^T from the
 //                 NVFP4 codes with the forward's block-scaled MMA (the same
@@ -25,17 +25,20 @@
 //                 over the first 32 columns of S, dQ^ += dS K^ with dS read
 //                 from TMEM; epilogue dq = c H (scale dQ^) in registers.
 //   bwd_kv_kernel one CTA per (head, 128 keys): per 64-query stage
-//                 S^T = K^Q^T and dP^T = V dO^T, P^T and dS^T as bf16 over
-//                 them, dV += P^T dO and dK^ += dS^T Q^ with A from TMEM;
+//                 S^T = K~Q~^T from the codes (block-scaled FP4 MMA) and
+//                 dP^T = V dO^T, P^T and dS^T as bf16 over the two halves of
+//                 S^T, dV += P^T dO and dK^ += dS^T Q^ with A from TMEM;
 //                 epilogue dv (bf16), scale dK^ (fp32 scratch) and each
 //                 warp's column sums of it (for the centring).
 //   colsum_kernel the head's column sums, added in a fixed order (so the
 //                 gradients are the same bits on every run).
 //   ste_k_kernel  one warp per key row: dk = c H (dK^ - colsum/N).
 // Warps: 0-3 compute (one TMEM lane = one row each), 4 the TMA producer, 5
-// the TMEM owner and MMA issuer.  TMEM (512 columns): X_b [64b, 64b+64) and
-// Y_b [128+64b, ...) for the two stage buffers b (S and dP, or S^T and dP^T),
-// accumulators at [256, 384) and [384, 512).  Every wait is bounded; a wait
+// the TMEM owner and MMA issuer.  TMEM (512 columns): stage buffers b at
+// [64b, 64b+64) for S (S^T); dQ kernel: dP_b at [128+64b, ...), dQ^ at
+// [256, 384), the scale factors at [384, 408); dK/dV kernel: one dP^T at
+// [128, 192), the scale factors at [192, 216), dV at [256, 384) and dK^ at
+// [384, 512).  Every wait is bounded; a wait
 // that runs out raises FP4ATTN_ERR_TIMEOUT and the CTA winds down.
 #include <cuda_bf16.h>
 
@@ -442,17 +445,27 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // ------------------------------------------------------- dK, dV kernel --
 
+// TMEM of the dK/dV kernel: S^T_b [64b, 64b+64) with P^T and dS^T written as
+// bf16 over its two halves, dP^T [128, 192) (one buffer: free once the compute
+// warps have loaded it), scale factors of K [192, 200) and two slots of Q's
+// [200, 208), [208, 216); dV [256, 384), dK^ [384, 512).
+constexpr uint32_t KV_DP = 128, KV_SFK = 192, KV_SFQ = 200;
+
 struct __align__(1024) KVSmem {
-    uint8_t k[TILE_R];                // K^ tile, K-major (A of S^T)
     uint8_t v[TILE_R];                // V tile, K-major (A of dP^T)
-    uint8_t q[STAGES][TILE_S];        // Q^ stage: K-major for S^T, MN-major for dK^ += dS^T Q^
+    uint8_t q[STAGES][TILE_S];        // Q~ stage (bf16): MN-major for dK^ += dS^T Q~
     uint8_t dout[STAGES][TILE_S];     // dO stage: K-major for dP^T, MN-major for dV += P^T dO
+    uint8_t kc[QC_BYTES];             // K codes (128 rows): A of S^T
+    uint8_t qc[STAGES][KC_BYTES];     // Q codes of the stage (64 rows): B of S^T
+    uint8_t ks_atom[2][512];          // scale-factor atoms for tcgen05.cp
+    uint8_t qs_atom[STAGES][2][512];
     float lse2[STAGES][BS];           // lse * log2(e) of the stage's queries (+inf past N)
     float dsum[STAGES][BS];           // D of the stage's queries (0 past N)
     uint64_t bar_kv_full;
     uint64_t bar_q_full[STAGES];
     uint64_t bar_q_empty[STAGES];
     uint64_t bar_s_full[2];
+    uint64_t bar_dp_free;             // the compute warps have loaded dP^T
     uint64_t bar_p_ready[2];
     uint64_t bar_final;
     uint32_t tmem_base;
@@ -482,9 +495,9 @@ __device__ __forceinline__ void warp_column_sums(float* a, int lane) {
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
-    bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p) {
+    bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     KVSmem& sm = *reinterpret_cast<KVSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
@@ -497,13 +510,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&sm.bar_kv_full), 1);
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&sm.bar_q_full[s]), 32);  // every producer lane (its lse / D stores)
+            mbar_init(smem_u32(&sm.bar_q_full[s]), 32);  // every producer lane (its lse / D / atom stores)
             mbar_init(smem_u32(&sm.bar_q_empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.bar_s_full[b]), 1);
             mbar_init(smem_u32(&sm.bar_p_ready[b]), 128);
         }
+        mbar_init(smem_u32(&sm.bar_dp_free), 128);
         mbar_init(smem_u32(&sm.bar_final), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -521,19 +535,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int hb = bh / p.H, hh = bh - hb * p.H;
 
     if (warp == WARP_PRODUCER) {
+        // K codes (with their scale atoms) and V once; per stage the Q codes and
+        // scale atoms, the bf16 Q~ and dO of BS queries, and their lse and D,
+        // all but the copies fetched one stage ahead
         const uint32_t kvf = smem_u32(&sm.bar_kv_full);
+        load_scale_atoms(p.k_scales + (size_t)bh * N + k0, N - k0, sm.ks_atom[0], sm.ks_atom[1], lane);
+        fence_proxy_async_smem();
+        __syncwarp();
         if (lane == 0) {
-            mbar_arrive_expect_tx(kvf, 2 * TILE_R);
-            tma_load_4d(smem_u32(sm.k), &tm_k, 0, k0, hh, hb, kvf);
-            tma_load_4d(smem_u32(sm.k) + PANEL_R, &tm_k, 64, k0, hh, hb, kvf);
+            mbar_arrive_expect_tx(kvf, QC_BYTES + TILE_R);
+            tma_load_3d(smem_u32(sm.kc), &tm_kc, 0, k0, bh, kvf);
             tma_load_4d(smem_u32(sm.v), &tm_v, 0, k0, hh, hb, kvf);
             tma_load_4d(smem_u32(sm.v) + PANEL_R, &tm_v, 64, k0, hh, hb, kvf);
         }
         const float* lse_head = p.lse + (size_t)bh * N;
         const float* d_head = p.dsum + (size_t)bh * N;
-        // lse and D of the next stage are loaded one stage ahead, so their
-        // latency overlaps the wait for a free buffer
+        const uint64_t* qs_head = p.q_scales + (size_t)bh * N;
         float nl[BS / 32], nd[BS / 32];
+        uint64_t qsc[4];
         auto fetch = [&](int i) {
 #pragma unroll
             for (int e = 0; e < BS / 32; ++e) {
@@ -541,6 +560,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 nl[e] = (qi < N) ? lse_head[qi] * kLog2e : INFINITY;
                 nd[e] = (qi < N) ? d_head[qi] : 0.0f;
             }
+            const int rest = N - i * BS;
+            fetch_scales(qs_head + i * BS, rest < BS ? rest : BS, lane, qsc);
         };
         fetch(0);
         int issued = 0;
@@ -554,11 +575,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 sm.lse2[st][lane + 32 * e] = nl[e];
                 sm.dsum[st][lane + 32 * e] = nd[e];
             }
+            store_scale_atoms(qsc, sm.qs_atom[st][0], sm.qs_atom[st][1], lane);
             if (i + 1 < T) fetch(i + 1);
+            fence_proxy_async_smem();
             const uint32_t full = smem_u32(&sm.bar_q_full[st]);
             if (lane == 0) {
                 const int r0 = i * BS;
-                mbar_arrive_expect_tx(full, 2 * TILE_S);
+                mbar_arrive_expect_tx(full, KC_BYTES + 2 * TILE_S);
+                tma_load_3d(smem_u32(sm.qc[st]), &tm_qc, 0, r0, bh, full);
                 tma_load_4d(smem_u32(sm.q[st]), &tm_q, 0, r0, hh, hb, full);
                 tma_load_4d(smem_u32(sm.q[st]) + PANEL_S, &tm_q, 64, r0, hh, hb, full);
                 tma_load_4d(smem_u32(sm.dout[st]), &tm_do, 0, r0, hh, hb, full);
@@ -576,39 +600,53 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         const bool leader = elect_one_sync();
-        const uint64_t kd = kmajor_desc(sm.k);
+        const uint64_t kcd = codes_desc(sm.kc, 0);
+        const uint64_t qcd0 = codes_desc(sm.qc[0], 0);      // stage st: + st * KC_BYTES / 16
+        const uint64_t qad0 = atom_desc(sm.qs_atom[0][0]);  // stage st: + 64 st, half h: + 32 h
         const uint64_t vd = kmajor_desc(sm.v);
-        const uint64_t qd0 = kmajor_desc(sm.q[0]);  // stage st: + st * TILE_S / 16
-        const uint64_t dod0 = kmajor_desc(sm.dout[0]);
+        const uint64_t dod0 = kmajor_desc(sm.dout[0]);      // stage st: + st * TILE_S / 16
         const uint64_t qmn0 = mn_desc(sm.q[0], PANEL_S);
         const uint64_t domn0 = mn_desc(sm.dout[0], PANEL_S);
-        constexpr uint64_t TD = TILE_S >> 4;
+        constexpr uint64_t TD = TILE_S >> 4, KCD = KC_BYTES >> 4, AD = (2 * 512) >> 4;
         auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort_flag, p.status, limit));
         };
-        auto scores = [&](int b, int st) {  // S^T_b = K^ Q^T, dP^T_b = V dO^T
+        // S^T_b = K~ Q~^T from the codes (Q scale factors of stage i into slot
+        // i & 1: the stage two back, which used that slot, was issued before)
+        auto scores = [&](int b, int st, int i) {
+            const uint32_t sfq = KV_SFQ + 8u * (uint32_t)(i & 1);
+            tmem_cp_32x128b_x4(tmem + sfq, qad0 + AD * st);
+            tmem_cp_32x128b_x4(tmem + sfq + 4, qad0 + AD * st + 32);
+            mma_mxf4nvf4(tmem + TM_X + BS * b, kcd, qcd0 + KCD * st, IDESC_S4, tmem + KV_SFK, tmem + sfq, 0u);
+            mma_mxf4nvf4(tmem + TM_X + BS * b, kcd + 2, qcd0 + KCD * st + 2, IDESC_S4, tmem + KV_SFK + 4,
+                         tmem + sfq + 4, 1u);
+        };
+        auto dprod = [&](int b, int st) {  // dP^T = V dO^T, then announce S^T_b and dP^T
 #pragma unroll
             for (int ks = 0; ks < 128 / 16; ++ks)
-                mma_bf16_ss(tmem + TM_X + BS * b, kd + kstep(PANEL_R, ks), qd0 + TD * st + kstep(PANEL_S, ks),
-                            IDESC_ST, ks > 0 ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < 128 / 16; ++ks)
-                mma_bf16_ss(tmem + TM_Y + BS * b, vd + kstep(PANEL_R, ks), dod0 + TD * st + kstep(PANEL_S, ks),
-                            IDESC_ST, ks > 0 ? 1u : 0u);
+                mma_bf16_ss(tmem + KV_DP, vd + kstep(PANEL_R, ks), dod0 + TD * st + kstep(PANEL_S, ks), IDESC_ST,
+                            ks > 0 ? 1u : 0u);
             tc_commit(smem_u32(&sm.bar_s_full[b]));
         };
-        auto accumulate = [&](int b, int st, bool acc) {  // dV += P^T dO, dK^ += dS^T Q^
+        auto accumulate = [&](int b, int st, bool acc) {  // dV += P^T dO, dK^ += dS^T Q~ (A from TMEM)
 #pragma unroll
             for (int ks = 0; ks < BS / 16; ++ks)
                 mma_bf16_ts(tmem + TM_ACC0, tmem + TM_X + BS * b + 8u * ks, domn0 + TD * st + MN_KSTEP * ks,
                             IDESC_AC, (acc || ks > 0) ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < BS / 16; ++ks)
-                mma_bf16_ts(tmem + TM_ACC1, tmem + TM_Y + BS * b + 8u * ks, qmn0 + TD * st + MN_KSTEP * ks,
+                mma_bf16_ts(tmem + TM_ACC1, tmem + TM_X + BS * b + 32u + 8u * ks, qmn0 + TD * st + MN_KSTEP * ks,
                             IDESC_AC, (acc || ks > 0) ? 1u : 0u);
             tc_commit(smem_u32(&sm.bar_q_empty[st]));
         };
         bool ok = wait(smem_u32(&sm.bar_kv_full), 0);
+        if (ok && leader) {
+            tc_fence_after();
+            const uint64_t kad = atom_desc(sm.ks_atom[0]);
+            tmem_cp_32x128b_x4(tmem + KV_SFK, kad);
+            tmem_cp_32x128b_x4(tmem + KV_SFK + 4, kad + 32);
+        }
+        __syncwarp();
         for (int i = 0; ok && i < T; ++i) {
             const int st = i % STAGES;
             if (!wait(smem_u32(&sm.bar_q_full[st]), (i / STAGES) & 1)) {
@@ -617,7 +655,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             if (leader) {
                 tc_fence_after();
-                scores(i & 1, st);
+                scores(i & 1, st, i);
+            }
+            __syncwarp();
+            // the single dP^T buffer: the compute warps must have loaded stage i-1's
+            if (i > 0 && !wait(smem_u32(&sm.bar_dp_free), (i - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            if (leader) {
+                tc_fence_after();
+                dprod(i & 1, st);
             }
             __syncwarp();
             if (i > 0) {
@@ -666,9 +714,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t sr[BS], dr[BS];
             tmem_ld32(tmem + lane_base + TM_X + BS * b, &sr[0]);
             tmem_ld32(tmem + lane_base + TM_X + BS * b + 32, &sr[32]);
-            tmem_ld32(tmem + lane_base + TM_Y + BS * b, &dr[0]);
-            tmem_ld32(tmem + lane_base + TM_Y + BS * b + 32, &dr[32]);
+            tmem_ld32(tmem + lane_base + KV_DP, &dr[0]);
+            tmem_ld32(tmem + lane_base + KV_DP + 32, &dr[32]);
             tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.bar_dp_free));  // dP^T may be overwritten
             const float4* l4 = reinterpret_cast<const float4*>(sm.lse2[st]);
             const float4* d4 = reinterpret_cast<const float4*>(sm.dsum[st]);
             uint32_t pk[BS / 2], dk[BS / 2];
@@ -688,8 +738,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
                 dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
             }
-            tmem_st32(tmem + lane_base + TM_X + BS * b, pk);  // P^T over S^T_b
-            tmem_st32(tmem + lane_base + TM_Y + BS * b, dk);  // dS^T over dP^T_b
+            tmem_st32(tmem + lane_base + TM_X + BS * b, pk);        // P^T over the first half of S^T_b
+            tmem_st32(tmem + lane_base + TM_X + BS * b + 32, dk);   // dS^T over its second half
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(smem_u32(&sm.bar_p_ready[b]));
@@ -824,12 +874,13 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     if (launch_dequant_bf16(a.q_codes, a.q_scales, nullptr, rows, a.qhat, stream) != cudaSuccess ||
         launch_dequant_bf16(a.k_codes, a.k_scales, nullptr, rows, a.khat, stream) != cudaSuccess)
         return FP4ATTN_ERR_CUDA;
-    CUtensorMap qc_r, kc_s, do_r, k_s, v_s, k_r, v_r, q_s, do_s;
+    CUtensorMap qc_r, kc_s, kc_r, qc_s, do_r, k_s, v_s, v_r, q_s, do_s;
     const Strides cs = contiguous_strides(a.H, a.N);  // Q~, K~: the library's own contiguous tensors
     if (!make_code_map(&qc_r, a.q_codes, a.BH, a.N, BR) || !make_code_map(&kc_s, a.k_codes, a.BH, a.N, BS) ||
+        !make_code_map(&kc_r, a.k_codes, a.BH, a.N, BR) || !make_code_map(&qc_s, a.q_codes, a.BH, a.N, BS) ||
         !make_map(&do_r, a.dout, B, a.H, a.N, BR, a.io) ||
         !make_map(&k_s, a.khat, B, a.H, a.N, BS, cs) || !make_map(&v_s, a.v, B, a.H, a.N, BS, a.io) ||
-        !make_map(&k_r, a.khat, B, a.H, a.N, BR, cs) || !make_map(&v_r, a.v, B, a.H, a.N, BR, a.io) ||
+        !make_map(&v_r, a.v, B, a.H, a.N, BR, a.io) ||
         !make_map(&q_s, a.qhat, B, a.H, a.N, BS, cs) || !make_map(&do_s, a.dout, B, a.H, a.N, BS, a.io))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(QSmem) + 1024 <= 227 * 1024, "shared memory budget");
@@ -866,7 +917,7 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     const dim3 grid((a.N + BR - 1) / BR, a.BH);
     bwd_q_kernel<<<grid, THREADS, smem_q, stream>>>(qc_r, do_r, kc_s, k_s, v_s, p);
     if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
-    bwd_kv_kernel<<<grid, THREADS, smem_kv, stream>>>(k_r, v_r, q_s, do_s, p);
+    bwd_kv_kernel<<<grid, THREADS, smem_kv, stream>>>(kc_r, v_r, qc_s, q_s, do_s, p);
     if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
     if (!(a.flags & FP4ATTN_NO_SMOOTH_K)) {
         colsum_kernel<<<a.BH, 128, 0, stream>>>(a.partial, 4 * (int)grid.x, a.colsum);
