@@ -26,20 +26,23 @@
 //                 from TMEM; epilogue dq = c H (scale dQ^) in registers.
 //   bwd_kv_kernel one CTA per (head, 128 keys): per 64-query stage
 //                 S^T = K~Q~^T from the codes (block-scaled FP4 MMA) and
-//                 dP^T = V dO^T, P^T and dS^T as bf16 over the two halves of
-//                 S^T, dV += P^T dO and dK^ += dS^T Q^ with A from TMEM;
+//                 dP^T = V dO^T, P^T and dS^T as bf16 over S^T (each compute
+//                 warp over the 32 columns it loaded), dV += P^T dO and
+//                 dK^ += dS^T Q^ with A from TMEM;
 //                 epilogue dv (bf16), scale dK^ (fp32 scratch) and each
 //                 warp's column sums of it (for the centring).
 //   colsum_kernel the head's column sums, added in a fixed order (so the
 //                 gradients are the same bits on every run).
 //   ste_k_kernel  one warp per key row: dk = c H (dK^ - colsum/N).
-// Warps: 0-3 compute (one TMEM lane = one row each), 4 the TMA producer, 5
-// the TMEM owner and MMA issuer.  TMEM (512 columns): stage buffers b at
-// [64b, 64b+64) for S (S^T); dQ kernel: dP_b at [128+64b, ...), dQ^ at
-// [256, 384), the scale factors at [384, 408); dK/dV kernel: one dP^T at
-// [128, 192), the scale factors at [192, 216), dV at [256, 384) and dK^ at
-// [384, 512).  Every wait is bounded; a wait
-// that runs out raises FP4ATTN_ERR_TIMEOUT and the CTA winds down.
+// Warps: the dQ kernel has 4 compute warps (one TMEM lane = one row each),
+// then the TMA producer and the TMEM owner / MMA issuer; the dK/dV kernel has
+// 8 compute warps (two per TMEM lane quarter, each taking half of a stage's
+// queries and half of the epilogue's columns), then the same two.  TMEM (512
+// columns): stage buffers b at [64b, 64b+64) for S (S^T); dQ kernel: dP_b at
+// [128+64b, ...), dQ^ at [256, 384), the scale factors at [384, 408); dK/dV
+// kernel: one dP^T at [128, 192), the scale factors at [192, 216), dV at
+// [256, 384) and dK^ at [384, 512).  Every wait is bounded; a wait that runs
+// out raises FP4ATTN_ERR_TIMEOUT and the CTA winds down.
 #include <cuda_bf16.h>
 
 #include "fp4_operands.cuh"
@@ -472,12 +475,12 @@ struct __align__(1024) KVSmem {
     int abort_flag;
 };
 
-// Sum of each of 128 columns over the 32 lanes of a warp: after five rounds of
+// Sum of each of NV columns over the 32 lanes of a warp: after five rounds of
 // exchanging half of the remaining partial sums, lane l holds the sums of
-// columns 4l .. 4l+3 in a[0..3].
-template <int R>
+// columns (NV/32)l .. (NV/32)l + NV/32 - 1 in a[0 .. NV/32 - 1].
+template <int NV, int R>
 __device__ __forceinline__ void column_sum_round(float* a, int lane) {
-    constexpr int half = 64 >> R;  // partial sums exchanged this round
+    constexpr int half = (NV / 2) >> R;  // partial sums exchanged this round
     const bool upper = (lane >> (4 - R)) & 1;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
@@ -486,15 +489,26 @@ __device__ __forceinline__ void column_sum_round(float* a, int lane) {
         a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16 >> R);
     }
 }
+template <int NV>
 __device__ __forceinline__ void warp_column_sums(float* a, int lane) {
-    column_sum_round<0>(a, lane);
-    column_sum_round<1>(a, lane);
-    column_sum_round<2>(a, lane);
-    column_sum_round<3>(a, lane);
-    column_sum_round<4>(a, lane);
+    column_sum_round<NV, 0>(a, lane);
+    column_sum_round<NV, 1>(a, lane);
+    column_sum_round<NV, 2>(a, lane);
+    column_sum_round<NV, 3>(a, lane);
+    column_sum_round<NV, 4>(a, lane);
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+// The dK/dV kernel's warps: 0-7 compute, 8 the TMA producer, 9 the MMA issuer.
+constexpr int KV_COMPUTE_WARPS = 8;
+constexpr int KV_THREADS = 32 * (KV_COMPUTE_WARPS + 2);
+constexpr int KV_WARP_PRODUCER = KV_COMPUTE_WARPS;
+constexpr int KV_WARP_MMA = KV_COMPUTE_WARPS + 1;
+// TMEM column (within S^T_b) of the bf16 P^T for K step ks (16 queries): the
+// compute warp of queries 32h .. writes P^T of them to columns 32h .. 32h+15
+// and dS^T to 32h+16 .. 32h+31.
+__host__ __device__ constexpr uint32_t kv_pcol(int ks) { return 32u * (uint32_t)(ks >> 1) + 8u * (uint32_t)(ks & 1); }
+
+__global__ void __launch_bounds__(KV_THREADS, 1)
     bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_v,
                   const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
@@ -515,14 +529,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.bar_s_full[b]), 1);
-            mbar_init(smem_u32(&sm.bar_p_ready[b]), 128);
+            mbar_init(smem_u32(&sm.bar_p_ready[b]), 32 * KV_COMPUTE_WARPS);
         }
-        mbar_init(smem_u32(&sm.bar_dp_free), 128);
+        mbar_init(smem_u32(&sm.bar_dp_free), 32 * KV_COMPUTE_WARPS);
         mbar_init(smem_u32(&sm.bar_final), 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == WARP_MMA) {
+    if (warp == KV_WARP_MMA) {
         tmem_alloc(smem_u32(&sm.tmem_base), TMEM_COLS);
         tmem_relinquish();
     }
@@ -534,7 +548,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint64_t limit = p.limit_ns;
     const int hb = bh / p.H, hh = bh - hb * p.H;
 
-    if (warp == WARP_PRODUCER) {
+    if (warp == KV_WARP_PRODUCER) {
         // K codes (with their scale atoms) and V once; per stage the Q codes and
         // scale atoms, the bf16 Q~ and dO of BS queries, and their lse and D,
         // all but the copies fetched one stage ahead
@@ -598,7 +612,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
                 drain_wait(smem_u32(&sm.bar_q_full[i % STAGES]), (i / STAGES) & 1);
         }
-    } else if (warp == WARP_MMA) {
+    } else if (warp == KV_WARP_MMA) {
         const bool leader = elect_one_sync();
         const uint64_t kcd = codes_desc(sm.kc, 0);
         const uint64_t qcd0 = codes_desc(sm.qc[0], 0);      // stage st: + st * KC_BYTES / 16
@@ -631,11 +645,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         auto accumulate = [&](int b, int st, bool acc) {  // dV += P^T dO, dK^ += dS^T Q~ (A from TMEM)
 #pragma unroll
             for (int ks = 0; ks < BS / 16; ++ks)
-                mma_bf16_ts(tmem + TM_ACC0, tmem + TM_X + BS * b + 8u * ks, domn0 + TD * st + MN_KSTEP * ks,
+                mma_bf16_ts(tmem + TM_ACC0, tmem + TM_X + BS * b + kv_pcol(ks), domn0 + TD * st + MN_KSTEP * ks,
                             IDESC_AC, (acc || ks > 0) ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < BS / 16; ++ks)
-                mma_bf16_ts(tmem + TM_ACC1, tmem + TM_X + BS * b + 32u + 8u * ks, qmn0 + TD * st + MN_KSTEP * ks,
+                mma_bf16_ts(tmem + TM_ACC1, tmem + TM_X + BS * b + kv_pcol(ks) + 16u, qmn0 + TD * st + MN_KSTEP * ks,
                             IDESC_AC, (acc || ks > 0) ? 1u : 0u);
             tc_commit(smem_u32(&sm.bar_q_empty[st]));
         };
@@ -694,9 +708,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ compute warps --
-        const int row = 32 * warp + lane;  // key row of the tile
+        // warps w and w+4 share TMEM lanes 32(w&3).. (key rows); warp half hc
+        // takes queries 32hc .. 32hc+31 of each stage and columns 64hc ..
+        // 64hc+63 of the epilogue
+        const int quarter = warp & 3, hc = warp >> 2;
+        const int row = 32 * quarter + lane;  // key row of the tile
         const int kn = k0 + row;
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         const float gq = p.gq ? *p.gq : 1.0f, gk = p.gk ? *p.gk : 1.0f;
         const float c = p.scale_log2 * gq * gk;  // S^T = scale gQ gK K~ Q~^T
         const float dk_scale = p.scale * gq;     // dK^ = scale dS^T Q^ = scale gQ dS^T Q~
@@ -711,19 +729,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t sr[BS], dr[BS];
-            tmem_ld32(tmem + lane_base + TM_X + BS * b, &sr[0]);
-            tmem_ld32(tmem + lane_base + TM_X + BS * b + 32, &sr[32]);
-            tmem_ld32(tmem + lane_base + KV_DP, &dr[0]);
-            tmem_ld32(tmem + lane_base + KV_DP + 32, &dr[32]);
+            const uint32_t own = TM_X + BS * b + 32u * hc;  // this warp's 32 columns of S^T_b
+            uint32_t sr[32], dr[32];
+            tmem_ld32(tmem + lane_base + own, sr);
+            tmem_ld32(tmem + lane_base + KV_DP + 32u * hc, dr);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&sm.bar_dp_free));  // dP^T may be overwritten
-            const float4* l4 = reinterpret_cast<const float4*>(sm.lse2[st]);
-            const float4* d4 = reinterpret_cast<const float4*>(sm.dsum[st]);
-            uint32_t pk[BS / 2], dk[BS / 2];
+            const float4* l4 = reinterpret_cast<const float4*>(sm.lse2[st] + 32 * hc);
+            const float4* d4 = reinterpret_cast<const float4*>(sm.dsum[st] + 32 * hc);
+            uint32_t pk[16], dk[16];
 #pragma unroll
-            for (int g = 0; g < BS / 4; ++g) {
+            for (int g = 0; g < 8; ++g) {
                 const float4 lv = l4[g], dv = d4[g];
                 const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
                 float pr[4], ds[4];
@@ -738,8 +755,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
                 dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
             }
-            tmem_st32(tmem + lane_base + TM_X + BS * b, pk);        // P^T over the first half of S^T_b
-            tmem_st32(tmem + lane_base + TM_X + BS * b + 32, dk);   // dS^T over its second half
+            // P^T and dS^T of these queries over the warp's own S^T columns
+            tmem_st16(tmem + lane_base + own, pk);
+            tmem_st16(tmem + lane_base + own + 16, dk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(smem_u32(&sm.bar_p_ready[b]));
@@ -748,15 +766,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const size_t grow = (size_t)bh * N + kn;
             const bool valid = kn < N;
-            // dV (bf16)
+            // dV (bf16), columns 64hc ..
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_base + TM_ACC0 + 32u * q, r);
+                const uint32_t col = 64u * hc + 32u * q;
+                tmem_ld32(tmem + lane_base + TM_ACC0 + col, r);
                 tmem_wait_ld();
                 if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(p.dv + row_offset(bh, p.H, kn, p.io_sb, p.io_sh, p.io_sn) +
-                                                          32 * q);
+                                                          col);
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
                         dst[v] = make_uint4(
@@ -766,31 +785,31 @@ __global__ void __launch_bounds__(THREADS, 1)
                             pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
                 }
             }
-            // scale * dK^ (fp32) and its column sums over the valid keys
-            float x[128];
+            // scale * dK^ (fp32) of columns 64hc .. and their sums over the valid keys
+            float x[64];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_base + TM_ACC1 + 32u * q, r);
+                tmem_ld32(tmem + lane_base + TM_ACC1 + 64u * hc + 32u * q, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[32 * q + e] = valid ? __uint_as_float(r[e]) * dk_scale : 0.0f;
             }
             if (valid) {
-                float4* dst = reinterpret_cast<float4*>(p.dk_acc + grow * 128);
+                float4* dst = reinterpret_cast<float4*>(p.dk_acc + grow * 128 + 64 * hc);
 #pragma unroll
-                for (int v = 0; v < 32; ++v) dst[v] = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+                for (int v = 0; v < 16; ++v) dst[v] = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
             }
-            warp_column_sums(x, lane);
-            float4* part = reinterpret_cast<float4*>(
-                p.partial + (((size_t)bh * gridDim.x + blockIdx.x) * 4 + warp) * 128);
-            part[lane] = make_float4(x[0], x[1], x[2], x[3]);
+            warp_column_sums<64>(x, lane);
+            float2* part = reinterpret_cast<float2*>(
+                p.partial + (((size_t)bh * gridDim.x + blockIdx.x) * 4 + quarter) * 128 + 64 * hc);
+            part[lane] = make_float2(x[0], x[1]);
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == WARP_MMA) {
+    if (warp == KV_WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -917,7 +936,7 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     const dim3 grid((a.N + BR - 1) / BR, a.BH);
     bwd_q_kernel<<<grid, THREADS, smem_q, stream>>>(qc_r, do_r, kc_s, k_s, v_s, p);
     if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
-    bwd_kv_kernel<<<grid, THREADS, smem_kv, stream>>>(kc_r, v_r, qc_s, q_s, do_s, p);
+    bwd_kv_kernel<<<grid, KV_THREADS, smem_kv, stream>>>(kc_r, v_r, qc_s, q_s, do_s, p);
     if (cudaGetLastError() != cudaSuccess) return FP4ATTN_ERR_CUDA;
     if (!(a.flags & FP4ATTN_NO_SMOOTH_K)) {
         colsum_kernel<<<a.BH, 128, 0, stream>>>(a.partial, 4 * (int)grid.x, a.colsum);
