@@ -449,9 +449,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 // ------------------------------------------------------- dK, dV kernel --
 
 // TMEM of the dK/dV kernel: S^T_b [64b, 64b+64) with P^T and dS^T written as
-// bf16 over its two halves, dP^T [128, 192) (one buffer: free once the compute
-// warps have loaded it), scale factors of K [192, 200) and two slots of Q's
-// [200, 208), [208, 216); dV [256, 384), dK^ [384, 512).
+// bf16 over it (each compute warp over the 32 columns it loaded), dP^T
+// [128, 192) (one buffer: free once the compute warps have loaded it), scale
+// factors of K [192, 200) and two slots of Q's [200, 208), [208, 216); dV
+// [256, 384), dK^ [384, 512).
 constexpr uint32_t KV_DP = 128, KV_SFK = 192, KV_SFQ = 200;
 
 struct __align__(1024) KVSmem {
