@@ -301,3 +301,88 @@ def attention_backward(q_codes, q_scales, k_codes, k_scales, v_bits, dO, gq=1.0,
                                                              None if O is None else O[b, h])
             out[0][b, h], out[1][b, h] = ste_grads(dqh, dkh, flags)
     return tuple(out)
+
+
+# -- sampled rows at full length ---------------------------------------------------
+
+def _bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def attention_all_rows(qhat: np.ndarray, khat: np.ndarray, v_bits: np.ndarray, scale=None, chunk: int = 1024):
+    """fp64 attention of every query row of one head at lengths where the
+    scalar C loop of attention_head is too slow (FastVideo "Pika H3 Flex in
+    FastVideo", section "FP4 attention": softmax(scale Q K^T) V over the
+    dequantised Q and K).  Each row is its own softmax, so rows are taken
+    `chunk` at a time, each by the plain definition (row max subtracted) with
+    torch's fp64 CPU matrix products and exponentials.  Inputs and outputs as
+    attention_head: (O [N,128] fp64, lse [N] fp64)."""
+    import torch
+
+    if scale is None:
+        scale = 1.0 / np.sqrt(128.0)
+    q = torch.from_numpy(np.ascontiguousarray(qhat, dtype=np.float32)).double()
+    kT = torch.from_numpy(np.ascontiguousarray(khat, dtype=np.float32)).double().T.contiguous()
+    v = torch.from_numpy(_bf16_bits_to_f64(v_bits))
+    N = q.shape[0]
+    O = torch.empty((N, 128), dtype=torch.float64)
+    lse = torch.empty((N,), dtype=torch.float64)
+    buf = torch.empty((min(chunk, N), kT.shape[1]), dtype=torch.float64)  # reused: no fresh pages per chunk
+    for r0 in range(0, N, chunk):
+        r1 = min(N, r0 + chunk)
+        s = buf[: r1 - r0]
+        torch.mm(q[r0:r1], kT, out=s)  # scores, then P in place
+        s.mul_(scale)
+        m = s.max(dim=1, keepdim=True).values
+        s.sub_(m).exp_()
+        l = s.sum(dim=1)
+        O[r0:r1] = (s @ v) / l[:, None]
+        lse[r0:r1] = m[:, 0] + torch.log(l)
+    return O.numpy(), lse.numpy()
+
+
+def attention_backward_rows(qhat: np.ndarray, khat: np.ndarray, v_bits: np.ndarray, dO: np.ndarray, O: np.ndarray,
+                            O_exact: np.ndarray, lse: np.ndarray, rows_q, rows_k, scale=None, flags: int = 0):
+    """Sampled rows of one head's training-time gradients -- what
+    attention_backward_head followed by ste_grads gives -- at lengths where
+    the N x N arrays are out of reach.  With P_ij = exp(scale qhat_i.khat_j -
+    lse_i), D_i = dO_i.O_i from the supplied forward output O, and
+    dS_ij = P_ij (dO_i.v_j - D_i):
+      query rows i:  dQ^_i = scale sum_j dS_ij khat_j,
+      key rows j:    dK^_j = scale sum_i dS_ij qhat_i,  dv_j = sum_i P_ij dO_i,
+    then dq = c H dQ^ and dk = c H (dK^ - mean_k dK^_k), as in ste_grads.
+    The key mean needs every row sum of dS; since the P_ij of a row sum to 1
+    and sum_j P_ij v_j is the exact output, sum_j dS_ij = dO_i.O_exact_i - D_i
+    (an exact rewrite of the sum), so the mean costs O(N d).  O_exact, lse:
+    the exact forward of attention_all_rows.  Returns (dq [|rows_q|,128],
+    dk [|rows_k|,128], dv [|rows_k|,128]), fp64."""
+    import torch
+
+    if scale is None:
+        scale = 1.0 / np.sqrt(128.0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    q = torch.from_numpy(np.ascontiguousarray(qhat, dtype=np.float32)).double()
+    k = torch.from_numpy(np.ascontiguousarray(khat, dtype=np.float32)).double()
+    v = torch.from_numpy(_bf16_bits_to_f64(v_bits))
+    g, Of, Oe, L = t(dO), t(O), t(O_exact), t(lse)
+    I = torch.from_numpy(np.asarray(rows_q, dtype=np.int64))
+    J = torch.from_numpy(np.asarray(rows_k, dtype=np.int64))
+    N = q.shape[0]
+    D = (g * Of).sum(dim=1)
+    # query rows
+    P = torch.exp((q[I] @ k.T) * scale - L[I][:, None])
+    dS = P * (g[I] @ v.T - D[I][:, None])
+    dqh = (dS @ k) * scale
+    # key rows (the transposed products)
+    PT = torch.exp((k[J] @ q.T) * scale - L[None, :])
+    dST = PT * (v[J] @ g.T - D[None, :])
+    dkh = (dST @ q) * scale
+    dv = PT @ g
+    if not flags & NO_SMOOTH_K:
+        rowsum = (g * Oe).sum(dim=1) - D
+        dkh = dkh - (rowsum @ q) * (scale / N)
+    # the rotation of ste_grads; the centring is done above
+    dq, _ = ste_grads(dqh.numpy(), np.zeros(dqh.shape), flags | NO_SMOOTH_K)
+    _, dk = ste_grads(np.zeros(dkh.shape), dkh.numpy(), flags | NO_SMOOTH_K)
+    return dq, dk, dv.numpy()

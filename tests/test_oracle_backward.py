@@ -171,3 +171,37 @@ def test_backward_with_given_output_equals_definition_at_the_exact_output():
         assert np.allclose(x, y, rtol=1e-11, atol=1e-13 * np.abs(x).max())
     c = oracle.attention_backward_head(q, k, vb, dO, O=O + 0.01)
     assert not np.allclose(c[0], a[0], rtol=1e-6) and np.array_equal(c[2], a[2])
+
+
+def test_attention_all_rows_equals_the_c_definition():
+    """The chunked fp64 forward (torch CPU ops) against the scalar C loop, with
+    a chunk size that leaves a ragged last chunk."""
+    q, k, vb, v, _ = _head(301, seed=41, k_bias=2.0)
+    O1, L1 = oracle.attention_head(q, k, vb)
+    O2, L2 = oracle.attention_all_rows(q, k, vb, chunk=64)
+    assert np.allclose(O2, O1, rtol=1e-12, atol=1e-14) and np.allclose(L2, L1, rtol=1e-13, atol=1e-13)
+    O3, L3 = oracle.attention_all_rows(q, k, vb, scale=0.05, chunk=1000)
+    O4, L4 = oracle.attention_head(q, k, vb, scale=0.05)
+    assert np.allclose(O3, O4, rtol=1e-12, atol=1e-14) and np.allclose(L3, L4, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("flags", [0, oracle.NO_SMOOTH_K, oracle.NO_HADAMARD, oracle.NO_SMOOTH_K | oracle.NO_HADAMARD])
+def test_sampled_backward_rows_equal_the_whole_head(flags):
+    """The sampled-row backward (the key mean through the row sums of dS) against
+    the whole-head C definition plus ste_grads, with D taken from a perturbed
+    forward output so that the rows of dS do not sum to zero."""
+    N = 257
+    q, k, vb, v, dO = _head(N, seed=43, k_bias=1.5)
+    O_exact, lse = oracle.attention_all_rows(q, k, vb)
+    O = O_exact + 0.01 * np.random.default_rng(2).standard_normal(O_exact.shape)
+    dqh, dkh, dv = oracle.attention_backward_head(q, k, vb, dO, O=O)
+    dq, dk = oracle.ste_grads(dqh, dkh, flags)
+    I = np.array([0, 5, 128, 256])
+    J = np.array([1, 17, 200, 256, 3])
+    a, b, c = oracle.attention_backward_rows(q, k, vb, dO, O, O_exact, lse, I, J, flags=flags)
+    for got, want in ((a, dq[I]), (b, dk[J]), (c, dv[J])):
+        assert np.allclose(got, want, rtol=1e-10, atol=1e-12 * np.abs(want).max())
+    # the centring term is not zero here, so dropping it would be caught
+    if not flags & oracle.NO_SMOOTH_K:
+        _, dk_raw = oracle.ste_grads(dqh, dkh, flags | oracle.NO_SMOOTH_K)
+        assert not np.allclose(b, dk_raw[J], rtol=1e-6, atol=0)
