@@ -6,8 +6,11 @@ binding) never imports it, and this package imports nothing from the product.
 
 It wraps the plain C implementation in ``oracle.c`` (codecs, exact fixed-point
 key mean, pinned-order Hadamard, NVFP4 pack, dequantisation and fp64
-attention) with numpy-friendly functions.  Every function is pinned by the CPU
-tests against something other than itself.
+attention) with numpy-friendly functions.  Two helpers for the longest
+sequences (every query row of a head's fp64 attention; sampled rows of the
+training-time gradients) use torch's fp64 CPU matrix products instead of the
+scalar C loops.  Every function is pinned by the CPU tests against something
+other than itself.
 
 Method source: FastVideo "Pika H3 Flex in FastVideo", section "FP4 attention"
 (smooth K, the same orthonormal Hadamard on Q and K, NVFP4 Q/K with E2M1 values
