@@ -166,3 +166,32 @@ def sample_rows(N: int, per_head: int, seed: int, tail_rows: int = 0, n_tail: in
     pool = np.setdiff1d(np.arange(N), np.fromiter(fixed, dtype=np.int64))
     extra = g.choice(pool, size=max(0, rest), replace=False) if rest > 0 else np.array([], dtype=np.int64)
     return np.sort(np.concatenate([np.fromiter(fixed, dtype=np.int64), extra.astype(np.int64)]))
+
+
+def toy_heads(n_heads: int, seed: int, N: int = 32, d: int = 64, k_bias_std: float = 2.0, n_scaled: int = 2,
+              scale_factor: float = 20.0) -> dict:
+    """The page's toy heads: ``d`` channels (64: four 16-value blocks), ``N``
+    keys and as many queries, Gaussian values, a per-channel key bias shared by
+    the keys of a head, and ``n_scaled`` channels scaled up in Q and K.
+
+    Same recipe as :func:`generate` with its own stream order: one
+    ``SeedSequence(seed)`` spawned into [bias and channels] + [Q] + [K] + [V];
+    the bias ``[n_heads, d] ~ N(0, k_bias_std^2)``, then the scaled channels
+    ``choice(d, n_scaled, replace=False)`` (shared by Q, K and every head),
+    then Q, K, V ``[n_heads, N, d]`` as float32 standard normals; scale the
+    channels, add the bias to K, cast to bf16 (round to nearest even).
+    Returns CPU bf16 tensors q, k, v ``[n_heads, N, d]`` and the channels."""
+    children = np.random.SeedSequence([seed, 64]).spawn(4)
+    g0 = np.random.Generator(np.random.PCG64(children[0]))
+    bias = (g0.standard_normal((n_heads, d)) * k_bias_std).astype(np.float32)
+    chans = np.sort(g0.choice(d, size=n_scaled, replace=False)) if n_scaled else np.array([], dtype=np.int64)
+    out = {}
+    for i, name in enumerate(("q", "k", "v")):
+        x = np.random.Generator(np.random.PCG64(children[1 + i])).standard_normal((n_heads, N, d), dtype=np.float32)
+        if name in ("q", "k") and n_scaled:
+            x[:, :, chans] *= np.float32(scale_factor)
+        if name == "k":
+            x += bias[:, None, :]
+        out[name] = torch.from_numpy(x).to(torch.bfloat16)
+    out["scaled_channels"] = chans
+    return out

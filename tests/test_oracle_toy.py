@@ -1,0 +1,119 @@
+"""The page's toy heads on the oracle (FastVideo "Pika H3 Flex in FastVideo",
+section "FP4 attention": 64 channels in four 16-value blocks, 32 keys,
+Gaussian values, a per-channel key bias and two scaled-up channels, NVFP4 Q
+and K at unit global scale, P and V in BF16).  The library's kernels are
+d = 128 only, so the toy runs on the oracle alone (CPU).
+
+Pins of the width-general restatement against things other than itself: the
+C oracle's 128-point transform and 128-channel prologue, scipy's Hadamard
+matrix, torch's fp64 attention, and the page's two exactness claims at d = 64.
+Then the toy study: FP4 with both transforms beats plain FP4, smoothing
+removes a key bias and the rotation spreads scaled channels."""
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+import oracle.toy as toy
+from nvfp4_precision_b200 import synth
+
+
+def _bits(t):
+    return synth.bf16_bits(t)
+
+
+def test_fwht_width_128_equals_the_c_transform_bit_for_bit():
+    x = np.random.default_rng(1).standard_normal((16, 128)).astype(np.float32) * 7
+    x[:, 5] *= 300
+    assert np.array_equal(toy.fwht(x), oracle.fwht128(x))
+
+
+def test_fwht_width_64_against_the_128_point_c_transform_and_scipy():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((16, 64)) * 5).astype(np.float32)
+    # H128 [x, x] = [2 H64 x, 0]: the first 32-stride stages of the 128-point
+    # transform are the 64-point ones on each half, then the halves are added
+    y128 = oracle.fwht128(np.concatenate([x, x], axis=1))
+    assert np.array_equal(y128[:, :64], 2 * toy.fwht(x)) and not y128[:, 64:].any()
+    H = scipy.linalg.hadamard(64).astype(np.float64)
+    xi = rng.integers(-1000, 1000, (8, 64)).astype(np.float32)
+    assert np.array_equal(toy.fwht(xi).astype(np.float64), xi.astype(np.float64) @ H)  # integers: exact
+    ref = x.astype(np.float64) @ H
+    assert np.abs(toy.fwht(x) - ref).max() <= 6 * 2.0 ** -24 * np.abs(x).sum(axis=1).max()
+
+
+def test_prologue_without_rotation_is_the_c_prologue_of_the_zero_padded_head():
+    t = synth.toy_heads(4, seed=3)
+    qb, kb = _bits(t["q"]), _bits(t["k"])
+    pad = lambda b: np.concatenate([b, np.zeros(b.shape, np.uint16)], axis=-1)
+    for flags in (oracle.NO_HADAMARD, oracle.NO_HADAMARD | oracle.NO_SMOOTH_K):
+        qh, kh = toy.prologue(qb, kb, flags)
+        ref = oracle.quantize_qk(pad(qb)[None], pad(kb)[None], flags=flags)
+        assert np.array_equal(qh, oracle.dequant(ref["q_codes"][0], ref["q_scales"][0])[..., :64])
+        assert np.array_equal(kh, oracle.dequant(ref["k_codes"][0], ref["k_scales"][0])[..., :64])
+
+
+def test_rotated_prologue_obeys_the_nvfp4_error_bound():
+    t = synth.toy_heads(8, seed=4)
+    qb, kb = _bits(t["q"]), _bits(t["k"])
+    qh, kh = toy.prologue(qb, kb, 0)
+    H = scipy.linalg.hadamard(64) / 8.0
+    k = synth.bf16_bits(t["k"])
+    kf = (k.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    kf = kf - kf.mean(axis=1, keepdims=True)
+    for exact, got in ((kf @ H, kh), (t["q"].double().numpy() @ H, qh)):
+        a = np.abs(exact).reshape(exact.shape[:-1] + (4, 16)).max(axis=-1, keepdims=True)
+        # block scale a/6 (rounded to E4M3, relative step 2^-3) and E2M1 steps of
+        # at most 2 scale units: a block's error is at most a/6 * (1 + 2^-3) * 1 + tiny
+        err = np.abs(got.astype(np.float64) - exact).reshape(a.shape[:-1] + (16,))
+        assert (err <= a / 6 * 1.13 + 1e-4 * a).all()
+
+
+def test_attention_matches_torch_and_bf16_p_stays_within_its_rounding():
+    t = synth.toy_heads(3, seed=5)
+    q, k = (t[n].double().numpy() for n in "qk")
+    vb = _bits(t["v"])
+    got = toy.attention(q, k, vb, bf16_p=False)
+    want = torch.nn.functional.scaled_dot_product_attention(t["q"].double(), t["k"].double(), t["v"].double())
+    assert np.allclose(got, want.numpy(), rtol=1e-12, atol=1e-13)
+    rounded = toy.attention(q, k, vb, bf16_p=True)
+    vmax = np.abs(t["v"].double().numpy()).max()
+    assert np.abs(rounded - got).max() <= 2.0 ** -8 * vmax
+
+
+def test_transforms_are_exact_before_quantisation_at_d64():
+    """(qH).(kH) = q.k and a shift shared by every key leaves softmax unchanged."""
+    t = synth.toy_heads(2, seed=6)
+    q, k = (t[n].double().numpy() for n in "qk")
+    H = scipy.linalg.hadamard(64) / 8.0
+    s = q @ np.swapaxes(k, 1, 2)
+    assert np.allclose((q @ H) @ np.swapaxes(k @ H, 1, 2), s, rtol=1e-12, atol=1e-9)
+    sm = lambda x: np.exp(x - x.max(-1, keepdims=True)) / np.exp(x - x.max(-1, keepdims=True)).sum(-1, keepdims=True)
+    ks = k - k.mean(axis=1, keepdims=True)
+    assert np.allclose(sm(q @ np.swapaxes(ks, 1, 2) / 8), sm(s / 8), rtol=1e-12, atol=1e-15)
+
+
+def _lower(e, better, worse="plain"):
+    """better's per-head error is below worse's: the mean paired difference
+    exceeds four standard errors (256 independent heads)."""
+    d = e[worse] - e[better]
+    return d.mean() > 4 * d.std(ddof=1) / np.sqrt(d.size)
+
+
+def test_toy_study_both_transforms_beat_plain_fp4():
+    t = synth.toy_heads(256, seed=7)
+    e = toy.errors(*(_bits(t[n]) for n in "qkv"))
+    print({k: round(float(v.mean()), 4) for k, v in e.items()})
+    assert _lower(e, "both")
+
+
+# The rotation's gain depends on how far the two channels are scaled (the page
+# gives no factor): clear at x10 with 32 keys, small at x20, reversed at x50.
+@pytest.mark.parametrize("kw,better", [(dict(n_scaled=0), "smooth K"),
+                                       (dict(k_bias_std=0.0, scale_factor=10.0), "Hadamard")])
+def test_each_transform_removes_the_error_it_targets(kw, better):
+    t = synth.toy_heads(256, seed=8, **kw)
+    e = toy.errors(*(_bits(t[n]) for n in "qkv"))
+    print(kw, {k: round(float(v.mean()), 4) for k, v in e.items()})
+    assert _lower(e, better)
