@@ -222,11 +222,12 @@ int fp4attn_quantize_qk_noalloc(const void* q_bf16_dev, const void* k_bf16_dev, 
  *   P = exp(scale Q^K^T - lse), dP = dO V^T, D = rowsum(dO * O),
  *   dS = P * (dP - D), dV = P^T dO, dQ^ = scale dS K^, dK^ = scale dS^T Q^,
  *   dq = c H dQ^, dk = c H (dK^ - mean_n dK^)   (c = 1/sqrt(128)).
- * The query-side kernel computes S from the codes with the forward's
- * block-scaled FP4 MMA (the scores the forward's lse was taken over); the
- * key-side kernel uses Q~, K~ in bf16 (exact), which this call dequantises
- * into the workspace.  P and dS are rounded to bf16 for the BF16 tensor-core
- * products, which accumulate in fp32; dq, dk, dv are bf16.  The global
+ * Both kernels compute their scores (S, and S^T on the key side) from the
+ * codes with the forward's block-scaled FP4 MMA (the scores the forward's lse
+ * was taken over); the products dQ^ += dS K~ and dK^ += dS^T Q~ take Q~, K~
+ * in bf16 (exact), which this call dequantises into the workspace.  P and dS
+ * are rounded to bf16 for the BF16 tensor-core products, which accumulate in
+ * fp32; dq, dk, dv are bf16.  The global
  * scales are applied as scalars (in the softmax scale and the dQ^ / dK^
  * factors), never by rounding gQ * Q~ to bf16.
  *   q_codes_dev, q_scales_dev, k_codes_dev, k_scales_dev : the forward's
