@@ -117,3 +117,10 @@ def test_each_transform_removes_the_error_it_targets(kw, better):
     e = toy.errors(*(_bits(t[n]) for n in "qkv"))
     print(kw, {k: round(float(v.mean()), 4) for k, v in e.items()})
     assert _lower(e, better)
+
+
+def test_bf16_rounding_of_p_equals_torch_cast():
+    x = np.random.default_rng(9).random(100000) * np.exp2(np.random.default_rng(10).integers(-30, 1, 100000))
+    x[:4] = [0.0, 1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8]  # ties: to even
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(toy._round_bf16(x), want)
