@@ -201,7 +201,10 @@ int fp4attn_forward_bf16qk_ex(const void* q_bf16_dev, fp4attn_strides q_strides,
  *     launch nothing;
  *   - the first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture;
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: after cudaDeviceReset (or anything else that tears down the
+ *     device's primary context) it is stale, so do not call this entry point
+ *     on that device again;
  *   - every call shares the one array and clears what must start at zero on
  *     its stream; calls that overlap on the GPU (other streams, other host
  *     threads) race on it and must be serialised by the caller. */

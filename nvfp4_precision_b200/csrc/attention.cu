@@ -30,7 +30,12 @@
 //     only moves when a stage's max exceeds it by more than 8 (so p <= 256),
 //     and only then is O_i rescaled in TMEM, after the previous P_i V has
 //     completed.  Exponentials are split between MUFU ex2 and a polynomial on
-//     the FMA pipe, with packed fp32x2 arithmetic.
+//     the FMA pipe, with packed fp32x2 arithmetic.  The row sum l is taken
+//     over the same bf16-rounded P that enters P V (each bf16 value widened
+//     exactly and added in fp32), so O / l is a convex combination of rows of
+//     V with the rounded weights: a row dominated by one key gets that key's
+//     V row back exactly, whatever the rounding of its p (which the lazy max
+//     leaves anywhere in (1, 256]).
 // Every wait is bounded; a wait that runs out raises FP4ATTN_ERR_TIMEOUT in
 // the status word and the CTA winds down (waiting for its own copies and MMAs)
 // instead of hanging.
@@ -500,8 +505,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                 } else {
                     pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                 }
-                lacc[k & 3] = __fadd2_rn(lacc[k & 3], pv);
                 pk[k] = pack_bf16x2(pv.x, pv.y);
+                lacc[k & 3] = add_bf16x2_to_f32x2(pk[k], lacc[k & 3]);
             }
             if (j > 0) {
                 // the previous P_i V has completed: its P buffer is free and O_i

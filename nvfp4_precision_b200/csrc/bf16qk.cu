@@ -25,7 +25,8 @@
 //     wait;
 //   * online softmax in the log2 domain with a lazy running max (it moves only
 //     when a stage's max exceeds it by more than 8, so p <= 256), exponentials
-//     split between MUFU ex2 and an FMA-pipe polynomial, packed fp32x2.
+//     split between MUFU ex2 and an FMA-pipe polynomial, packed fp32x2; the
+//     row sum is taken over the same bf16-rounded P that enters P V.
 // Every wait is bounded; a wait that runs out raises FP4ATTN_ERR_TIMEOUT in the
 // status word and the CTA winds down instead of hanging.
 #include <cuda_bf16.h>
@@ -353,8 +354,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 } else {
                     pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                 }
-                lacc[k & 3] = __fadd2_rn(lacc[k & 3], pv);
                 pk[k] = pack_bf16x2(pv.x, pv.y);
+                lacc[k & 3] = add_bf16x2_to_f32x2(pk[k], lacc[k & 3]);
             }
             // P (bf16 pairs) over the first 64 columns of S_i
             tmem_st32(s_addr, &pk[0]);

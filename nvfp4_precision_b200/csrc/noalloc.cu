@@ -33,7 +33,10 @@ std::mutex g_mutex;
 void* g_scratch_dev[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached for the life of the
+// process.  The cache does not survive a teardown of the device's primary
+// context (cudaDeviceReset): the module, and the array with it, may then be
+// loaded at another address.
 int scratch_on_current_device(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -410,6 +410,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// acc + (the two bf16 values of w, each widened exactly), one rounding each:
+// the row sum of P taken over the very bf16 values the P V product uses.
+__device__ __forceinline__ float2 add_bf16x2_to_f32x2(uint32_t w, float2 acc) {
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(w));
+    return acc;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -65,3 +65,28 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     rc = fa.lib.fp4attn_quantize_qk_noalloc(ptr, ptr, fa.Shape(32, 33, 128, 128), None, None, 0,
                                             ptr, ptr, ptr, ptr, None, None, None)
     assert rc == fa.ERR_UNSUPPORTED
+
+
+def test_noalloc_device_errors_reach_the_status_word_and_are_cleared_by_the_next_call():
+    """The shared scratch keeps the last call's contents, so each call must
+    clear its status word: a call with a non-finite global scale reports
+    FP4ATTN_ERR_RANGE through status_dev, and the good call after it reports 0.
+    An empty shape (N = 0) launches nothing and also reports 0."""
+    fa = _fa()
+    q, k = _inputs("err", 1, 2, 256, 5)
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    bad = torch.tensor([float("inf")], dtype=torch.float32, device="cuda")
+    fa.fp4attn_quantize_qk_noalloc(q, k, bad, None, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == fa.ERR_RANGE
+    ref = fa.fp4attn_quantize_qk(q, k)
+    got = fa.fp4attn_quantize_qk_noalloc(q, k, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for key in KEYS:
+        assert torch.equal(got[key], ref[key]), f"after an error: {key} differs"
+    fa.fp4attn_quantize_qk_noalloc(q, k, bad, None, status=status)
+    e = torch.empty((1, 2, 0, 128), dtype=torch.bfloat16, device="cuda")
+    fa.fp4attn_quantize_qk_noalloc(e, e, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
