@@ -324,6 +324,20 @@ int fp4attn_probe_div6(uint32_t* result_dev, cudaStream_t stream);
  * FP4ATTN_ERR_TIMEOUT into *status_dev (device int32, set to 0 first). */
 int fp4attn_probe_wait_timeout(int* status_dev, uint64_t limit_ns, cudaStream_t stream);
 
+/* Runs fp4attn_quantize_qk on contiguous Q and K with the key-sum tiles
+ * withheld, so the first K tile of every head waits for column sums that no
+ * tile computes.  That wait must give up after limit_ns (at most 10 s), write
+ * FP4ATTN_ERR_TIMEOUT into the workspace status word and let every CTA wind
+ * down (each waits for its own copies in flight) and return.  Arguments as
+ * fp4attn_quantize_qk without the global scales, flags and key mean; the
+ * workspace is cleared first.  Q codes and scales are written as usual; the
+ * K outputs are unspecified. */
+int fp4attn_probe_withheld_key_sums(const void* q_bf16_dev, const void* k_bf16_dev, fp4attn_shape s,
+                                    uint8_t* q_codes_dev, uint8_t* q_scales_dev,
+                                    uint8_t* k_codes_dev, uint8_t* k_scales_dev,
+                                    void* workspace_dev, size_t workspace_bytes, uint64_t limit_ns,
+                                    cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

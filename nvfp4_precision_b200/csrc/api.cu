@@ -412,4 +412,36 @@ int fp4attn_probe_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t stre
     return launch_probe_wait_timeout(status, limit_ns, stream);
 }
 
+int fp4attn_probe_withheld_key_sums(const void* q, const void* k, fp4attn_shape s, uint8_t* q_codes,
+                                    uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales, void* workspace,
+                                    size_t workspace_bytes, uint64_t limit_ns, cudaStream_t stream) {
+    int st = check_shape(s);
+    if (st != FP4ATTN_OK) return st;
+    if (empty(s) || limit_ns > 10000000000ull) return FP4ATTN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
+        return FP4ATTN_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, q_codes, q_scales, k_codes, k_scales};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return FP4ATTN_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, fp4attn_workspace_bytes(s), stream);
+    if (e != cudaSuccess) return launch_status(e);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    QuantArgs a{};
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.qs = a.ks = contiguous_strides(s.H, s.N);
+    a.BH = (int)heads(s);
+    a.H = s.H;
+    a.N = s.N;
+    a.q_codes = q_codes;
+    a.q_scales = q_scales;
+    a.k_codes = k_codes;
+    a.k_scales = k_scales;
+    a.ksum = reinterpret_cast<long long*>(ws + ws_ksum_offset());
+    a.counters = reinterpret_cast<unsigned*>(ws + ws_counter_offset(heads(s)));
+    a.ticket = reinterpret_cast<unsigned*>(ws + WS_TICKET_OFFSET);
+    a.status = reinterpret_cast<int*>(ws);
+    return launch_status(launch_quantize_qk_withheld_sums(a, limit_ns, stream));
+}
+
 }  // extern "C"

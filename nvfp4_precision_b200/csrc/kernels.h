@@ -57,6 +57,8 @@ struct QuantArgs {
 };
 
 cudaError_t launch_quantize_qk(const QuantArgs& a, cudaStream_t stream);
+// Test hook: the prologue with its key-sum tiles withheld (K tiles time out).
+cudaError_t launch_quantize_qk_withheld_sums(const QuantArgs& a, uint64_t spin_limit_ns, cudaStream_t stream);
 // Dynamic global scales of empty tensors (amax 0): store the smallest g, 2^-64.
 cudaError_t launch_store_gscales(float* gq, float* gk, cudaStream_t stream);
 

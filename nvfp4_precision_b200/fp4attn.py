@@ -34,6 +34,7 @@ EXPORTS = (
     "fp4attn_backward_workspace_bytes",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout", "fp4attn_probe_div6",
+    "fp4attn_probe_withheld_key_sums",
 )
 
 
@@ -105,6 +106,8 @@ def _load():
     L.fp4attn_probe_div6.argtypes = [P, P]
     L.fp4attn_probe_wait_timeout.restype = ctypes.c_int
     L.fp4attn_probe_wait_timeout.argtypes = [P, U64, P]
+    L.fp4attn_probe_withheld_key_sums.restype = ctypes.c_int
+    L.fp4attn_probe_withheld_key_sums.argtypes = [P, P, Shape, P, P, P, P, P, ctypes.c_size_t, U64, P]
     return L
 
 
@@ -408,3 +411,21 @@ def fp4attn_probe_wait_timeout(limit_ns: int, stream=None) -> int:
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     _check(lib.fp4attn_probe_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)), "fp4attn_probe_wait_timeout")
     return int(status.item())
+
+
+def fp4attn_probe_withheld_key_sums(q: torch.Tensor, k: torch.Tensor, limit_ns: int, stream=None) -> int:
+    """The prologue with its key-sum tiles withheld: returns the device status
+    after the run (FP4ATTN_ERR_TIMEOUT when the K tiles' bounded wait gave up)."""
+    assert q.dtype == torch.bfloat16 and k.dtype == torch.bfloat16 and q.shape == k.shape
+    assert q.is_contiguous() and k.is_contiguous()
+    B, H, N, D = q.shape
+    dev = q.device
+    qc = torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev)
+    qs = torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev)
+    kc = torch.empty_like(qc)
+    ks = torch.empty_like(qs)
+    ws = new_workspace(B, H, N)
+    _check(lib.fp4attn_probe_withheld_key_sums(_ptr(q), _ptr(k), Shape(B, H, N, D), _ptr(qc), _ptr(qs), _ptr(kc),
+                                               _ptr(ks), _ptr(ws), ws.numel(), int(limit_ns), _stream(stream)),
+           "fp4attn_probe_withheld_key_sums")
+    return fp4attn_read_status(ws)

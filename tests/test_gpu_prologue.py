@@ -132,3 +132,16 @@ def test_empty_shapes_are_no_ops():
     q = torch.zeros((2, 3, 0, 128), dtype=torch.bfloat16, device="cuda")
     out = fa().fp4attn_quantize_qk(q, q)
     assert out["q_codes"].numel() == 0
+
+
+def test_withheld_key_sums_time_out_and_the_kernel_returns():
+    """Failure detection without a GPU fault: the prologue runs with its
+    key-sum tiles withheld, so every head's K tiles wait for column sums that
+    never arrive.  The wait is bounded (1 ms here): the status word must read
+    FP4ATTN_ERR_TIMEOUT, the kernel must return, and the context must stay
+    usable -- the ordinary prologue right after it is still bit-exact."""
+    d = synth.generate(synth.custom("withheld", 1, 3, 1000, seed=11, k_offset_std=2.0), ("q", "k"))
+    q, k = d["q"].cuda(), d["k"].cuda()
+    assert fa().fp4attn_probe_withheld_key_sums(q, k, 1_000_000) == fa().ERR_TIMEOUT
+    torch.cuda.synchronize()
+    assert_prologue_equal(gpu_prologue(d), oracle_prologue(d), "after a timed-out launch")
