@@ -67,7 +67,7 @@
 #define FP4ATTN_PRO_CTAS 1     // resident CTAs per SM the kernel is built for
 #endif
 #ifndef FP4ATTN_PRO_RUN
-#define FP4ATTN_PRO_RUN 8      // consecutive tiles per ticket request
+#define FP4ATTN_PRO_RUN 8      // most consecutive tiles per ticket request
 #endif
 #ifndef FP4ATTN_PRO_LEAD
 #define FP4ATTN_PRO_LEAD 1     // key sums of head h+1 between Q(h) and K(h)
@@ -85,7 +85,7 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr int W = FP4ATTN_PRO_W;
 constexpr int NSLOT = FP4ATTN_PRO_NSLOT;
 constexpr int CTAS_PER_SM = FP4ATTN_PRO_CTAS;
-constexpr int TICKET_RUN = FP4ATTN_PRO_RUN;
+constexpr int MAX_TICKET_RUN = FP4ATTN_PRO_RUN;
 constexpr int PRO_THREADS = 32 * (W + 1);
 constexpr int TILE_ROWS = 16 * W;
 constexpr uint32_t HALF_BYTES = TILE_ROWS * 128;  // TILE_ROWS rows x 64 channels bf16
@@ -122,6 +122,7 @@ struct ProArgs {
     bool sums_ready;   // the key sums of every head are complete: no key-sum tiles
     bool withhold_sums;  // test hook: K tiles wait for key sums that no tile computes
     int lead;          // 1: key sums of head h+1 between Q(h) and K(h); 0: ahead of Q(h)
+    int run;           // consecutive tiles per ticket request
     uint64_t spin_limit_ns;
     int* status;
 };
@@ -296,19 +297,20 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             const uint64_t pol_keep = l2_policy_evict_last();
             const uint64_t pol_stream = l2_policy_evict_first();
             uint32_t filled = 0u, parity = 0u;  // per slot: ever filled; parity of its last fill
-            // tickets come in runs of TICKET_RUN consecutive tiles, the next
+            // tickets come in runs of a.run consecutive tiles, the next
             // run requested as soon as the current one starts, so the
             // atomic's round trip overlaps the fills instead of preceding each
-            int run = (int)atomicAdd(a.ticket, (unsigned)TICKET_RUN);
-            int run_next = (int)atomicAdd(a.ticket, (unsigned)TICKET_RUN);
+            const int run_len = a.run;
+            int run = (int)atomicAdd(a.ticket, (unsigned)run_len);
+            int run_next = (int)atomicAdd(a.ticket, (unsigned)run_len);
             int in_run = 0;
             for (int i = 0;; ++i) {
                 const int s = i % NSLOT;
                 const uint32_t ph = (uint32_t)(i / NSLOT) & 1u;
-                if (in_run == TICKET_RUN) {
+                if (in_run == run_len) {
                     run = run_next;
                     in_run = 0;
-                    if (run < total) run_next = (int)atomicAdd(a.ticket, (unsigned)TICKET_RUN);
+                    if (run < total) run_next = (int)atomicAdd(a.ticket, (unsigned)run_len);
                 }
                 const int t = run + in_run++;
 #ifdef FP4ATTN_PRO_SPIN
@@ -724,6 +726,13 @@ ProArgs base_args(const QuantArgs& q) {
     a.n_tiles = (q.N + TILE_ROWS - 1) / TILE_ROWS;
     a.flags = q.flags & ~QUANT_DYNAMIC_G;
     a.lead = FP4ATTN_PRO_LEAD;
+    // The tiles taken but not yet finished across the GPU (the CTAs' rings plus
+    // two ticket runs each) must stay well below the distance from a head's
+    // key-sum tiles to its K tiles (three runs of n_tiles), or K tiles wait:
+    // runs of about n_tiles / 48 tiles, 1 to MAX_TICKET_RUN.
+    a.run = a.n_tiles / 48;
+    if (a.run < 1) a.run = 1;
+    if (a.run > MAX_TICKET_RUN) a.run = MAX_TICKET_RUN;
     a.spin_limit_ns = kWaitLimitNs;
     a.status = q.status;
     return a;
