@@ -35,6 +35,14 @@
  *   k_mean       fp32  [B, H, 128]
  *   O            bf16  [B, H, N, 128]
  *   lse          fp32  [B, H, N]       natural-log sum of exp of the scaled logits
+ * Heads of D = 64 channels (the page's toy heads: section "FP4 attention",
+ * 64 channels in four 16-value blocks) are taken by fp4attn_quantize_qk,
+ * fp4attn_quantize_qk_ex (static global scales), fp4attn_forward,
+ * fp4attn_forward_ex and the dequantisers: Q, K, V and O are [B, H, N, 64],
+ * codes [B, H, N, 32], scales [B, H, N, 4], k_mean [B, H, 64]; the rotation
+ * is the 64-point transform (six butterfly stages) times fp32(1/sqrt(64)),
+ * and softmax_scale <= 0 selects 1/sqrt(64).  The other entry points take
+ * D = 128 only.
  * Every pointer must be 16-byte aligned.  Pointers named *_dev are device
  * pointers (cudaMalloc / torch CUDA tensors); none may alias another output.
  *
@@ -58,7 +66,7 @@ extern "C" {
 typedef enum {
     FP4ATTN_OK = 0,
     FP4ATTN_ERR_INVALID_ARG = 1,  /* bad shape, NULL or misaligned pointer      */
-    FP4ATTN_ERR_UNSUPPORTED = 2,  /* valid but not supported (e.g. D != 128)    */
+    FP4ATTN_ERR_UNSUPPORTED = 2,  /* valid but not supported (e.g. D = 96)      */
     FP4ATTN_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed          */
     FP4ATTN_ERR_RANGE = 4,        /* device: non-finite input, |k| >= 2^20, g<=0 */
     FP4ATTN_ERR_TIMEOUT = 5,      /* device: a bounded wait ran out             */
@@ -76,10 +84,10 @@ enum {
 };
 
 typedef struct {
-    int32_t B, H, N, D;  /* D must be 128; B, H, N >= 0; N <= 262144 */
+    int32_t B, H, N, D;  /* D = 128 (or 64 where stated); B, H, N >= 0; N <= 262144 */
 } fp4attn_shape;
 
-/* Element strides of a bf16 tensor indexed [b][h][n][c] (c, the 128 channels,
+/* Element strides of a bf16 tensor indexed [b][h][n][c] (c, the D channels,
  * always contiguous).  Each stride must be a positive multiple of 8 elements
  * (16 bytes) below 2^39; the stride of a dimension of size 1 is ignored.  The
  * contiguous [B,H,N,128] layout is {H*N*128, N*128, 128}; a [B,N,H,128]
@@ -114,7 +122,8 @@ int fp4attn_quantize_qk(const void* q_bf16_dev, const void* k_bf16_dev, fp4attn_
 /* fp4attn_quantize_qk for Q and K of any strides (fp4attn_strides), with an
  * optional dynamic global scale.  The codes, scales and k_mean outputs keep the
  * layouts of fp4attn_quantize_qk.
- *   flags : as for fp4attn_quantize_qk, plus FP4ATTN_DYNAMIC_GSCALE.
+ *   flags : as for fp4attn_quantize_qk, plus FP4ATTN_DYNAMIC_GSCALE (D = 128
+ *     only; FP4ATTN_ERR_UNSUPPORTED for D = 64).
  *   q_gscale_dev, k_gscale_dev : without FP4ATTN_DYNAMIC_GSCALE, inputs as for
  *     fp4attn_quantize_qk (NULL for 1.0).  With it, both must be non-NULL and
  *     receive g = fl32(amax / (6 * 448)), raised to 2^-64 when smaller, where
@@ -138,7 +147,7 @@ int fp4attn_quantize_qk_ex(const void* q_bf16_dev, fp4attn_strides q_strides,
  *   O = softmax(scale * gQ * gK * (Qc K c^T)) V,  Qc, Kc the block-scaled E2M1
  *   values; Q K^T on the FP4 tensor cores with fp32 accumulation, P rounded to
  *   bf16 for P.V, fp32 accumulation, online softmax.
- *   softmax_scale : <= 0 selects 1/sqrt(128).
+ *   softmax_scale : <= 0 selects 1/sqrt(D).
  *   o_bf16_dev : [B,H,N,128] out.  lse_dev : [B,H,N] out or NULL.
  *   workspace_dev : as for fp4attn_quantize_qk (status word only; not cleared).
  * Device errors: FP4ATTN_ERR_RANGE for a bad g; FP4ATTN_ERR_TIMEOUT if an
@@ -167,7 +176,7 @@ int fp4attn_forward_ex(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev,
  * tensor cores with fp32 accumulation; softmax, P (bf16) and P V are as in
  * fp4attn_forward.  No smoothing, rotation or quantisation is applied.
  *   q_bf16_dev, k_bf16_dev, v_bf16_dev : [B,H,N,128] bf16.
- *   softmax_scale : <= 0 selects 1/sqrt(128).
+ *   softmax_scale : <= 0 selects 1/sqrt(D).
  *   o_bf16_dev : [B,H,N,128] out.  lse_dev : [B,H,N] out or NULL.
  *   workspace_dev : as for fp4attn_forward (status word only; not cleared).
  * Device errors: FP4ATTN_ERR_TIMEOUT if an internal wait ran out. */

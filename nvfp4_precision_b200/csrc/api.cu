@@ -19,9 +19,10 @@ constexpr int32_t kMaxN = 262144;  // 2^18: keeps |sum of k * 2^24| < 2^62 for |
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_shape(fp4attn_shape s) {
+// d = 128, or 64 for the entry points that take narrow heads (allow64)
+int check_shape(fp4attn_shape s, bool allow64 = false) {
     if (s.B < 0 || s.H < 0 || s.N < 0 || s.D <= 0) return FP4ATTN_ERR_INVALID_ARG;
-    if (s.D != D) return FP4ATTN_ERR_UNSUPPORTED;
+    if (s.D != D && !(allow64 && s.D == 64)) return FP4ATTN_ERR_UNSUPPORTED;
     if (s.N > kMaxN) return FP4ATTN_ERR_UNSUPPORTED;
     const int64_t bh = (int64_t)s.B * s.H;
     if (bh > 65535 || bh * (int64_t)s.N >= ((int64_t)1 << 31)) return FP4ATTN_ERR_UNSUPPORTED;
@@ -30,11 +31,11 @@ int check_shape(fp4attn_shape s) {
 
 int64_t heads(fp4attn_shape s) { return (int64_t)s.B * s.H; }
 
-// Strides of a [B,H,N,128] bf16 tensor: positive multiples of 8 elements
+// Strides of a [B,H,N,D] bf16 tensor: positive multiples of 8 elements
 // (16 bytes, the tensor-copy rule) below 2^39 elements (2^40 bytes); a
 // dimension of size 1 takes the contiguous stride instead of the caller's.
 bool normalise_strides(fp4attn_shape s, fp4attn_strides in, Strides* out) {
-    const Strides c = contiguous_strides(s.H, s.N);
+    const Strides c = contiguous_strides(s.H, s.N, s.D);
     const int64_t v[3] = {s.B == 1 ? c.b : in.b, s.H == 1 ? c.h : in.h, s.N == 1 ? c.n : in.n};
     for (int64_t x : v)
         if (x <= 0 || (x & 7) || x >= ((int64_t)1 << 39)) return false;
@@ -43,7 +44,7 @@ bool normalise_strides(fp4attn_shape s, fp4attn_strides in, Strides* out) {
 }
 
 fp4attn_strides contiguous(fp4attn_shape s) {
-    const Strides c = contiguous_strides(s.H, s.N);
+    const Strides c = contiguous_strides(s.H, s.N, s.D);
     return fp4attn_strides{c.b, c.h, c.n};
 }
 bool empty(fp4attn_shape s) { return heads(s) == 0 || s.N == 0; }
@@ -113,11 +114,12 @@ int fp4attn_quantize_qk_ex(const void* q, fp4attn_strides q_strides, const void*
                            fp4attn_shape s, float* gq, float* gk, uint32_t flags, uint8_t* q_codes,
                            uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales, float* k_mean,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-    int st = check_shape(s);
+    int st = check_shape(s, true);
     if (st != FP4ATTN_OK) return st;
     if (flags & ~(uint32_t)(FP4ATTN_NO_SMOOTH_K | FP4ATTN_NO_HADAMARD | FP4ATTN_DYNAMIC_GSCALE))
         return FP4ATTN_ERR_INVALID_ARG;
     const bool dynamic = (flags & FP4ATTN_DYNAMIC_GSCALE) != 0;
+    if (dynamic && s.D != D) return FP4ATTN_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
         return FP4ATTN_ERR_WORKSPACE;
     if ((gq && ((uintptr_t)gq & 3)) || (gk && ((uintptr_t)gk & 3))) return FP4ATTN_ERR_INVALID_ARG;
@@ -135,6 +137,27 @@ int fp4attn_quantize_qk_ex(const void* q, fp4attn_strides q_strides, const void*
     if (e != cudaSuccess) return launch_status(e);
     if (empty(s)) return dynamic ? launch_status(launch_store_gscales(gq, gk, stream)) : FP4ATTN_OK;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (s.D == 64) {
+        Prologue64Args b{};
+        b.q = static_cast<const __nv_bfloat16*>(q);
+        b.k = static_cast<const __nv_bfloat16*>(k);
+        b.qs = qs;
+        b.ks = ks;
+        b.BH = (int)heads(s);
+        b.H = s.H;
+        b.N = s.N;
+        b.flags = flags;
+        b.gq = gq;
+        b.gk = gk;
+        b.q_codes = q_codes;
+        b.q_scales = q_scales;
+        b.k_codes = k_codes;
+        b.k_scales = k_scales;
+        b.k_mean = k_mean;
+        b.ksum = reinterpret_cast<long long*>(ws + ws_ksum_offset());
+        b.status = reinterpret_cast<int*>(ws);
+        return launch_status(launch_quantize_qk64(b, stream));
+    }
     QuantArgs a;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.k = static_cast<const __nv_bfloat16*>(k);
@@ -175,7 +198,7 @@ int fp4attn_forward_ex(const uint8_t* q_codes, const uint8_t* q_scales, const ui
                        fp4attn_strides v_strides, fp4attn_shape s, float softmax_scale, void* o,
                        fp4attn_strides o_strides, float* lse, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream) {
-    int st = check_shape(s);
+    int st = check_shape(s, true);
     if (st != FP4ATTN_OK) return st;
     if (!workspace || workspace_bytes < fp4attn_workspace_bytes(s) || !aligned16(workspace))
         return FP4ATTN_ERR_WORKSPACE;
@@ -198,6 +221,7 @@ int fp4attn_forward_ex(const uint8_t* q_codes, const uint8_t* q_scales, const ui
     a.v = static_cast<const __nv_bfloat16*>(v);
     a.BH = (int)heads(s);
     a.N = s.N;
+    a.d = s.D;
     a.softmax_scale = softmax_scale;
     a.o = static_cast<__nv_bfloat16*>(o);
     a.lse = lse;
@@ -326,24 +350,26 @@ int fp4attn_backward(const uint8_t* q_codes, const uint8_t* q_scales, const uint
 
 int fp4attn_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s, void* out,
                          cudaStream_t stream) {
-    int st = check_shape(s);
+    int st = check_shape(s, true);
     if (st != FP4ATTN_OK) return st;
     if (empty(s)) return FP4ATTN_OK;
-    if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out) || ((uintptr_t)scales & 7))
+    if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out) ||
+        ((uintptr_t)scales & (uintptr_t)(s.D / 16 - 1)))  // a row's scales: 8 bytes (4 for 64 channels)
         return FP4ATTN_ERR_INVALID_ARG;
     if (g && ((uintptr_t)g & 3)) return FP4ATTN_ERR_INVALID_ARG;
-    return launch_status(
-        launch_dequant_bf16(codes, scales, g, heads(s) * s.N, static_cast<__nv_bfloat16*>(out), stream));
+    return launch_status(launch_dequant_bf16(codes, scales, g, heads(s) * s.N * (s.D / 16),
+                                             static_cast<__nv_bfloat16*>(out), stream));
 }
 
 int fp4attn_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, fp4attn_shape s,
                     float* out, cudaStream_t stream) {
-    int st = check_shape(s);
+    int st = check_shape(s, true);
     if (st != FP4ATTN_OK) return st;
     if (empty(s)) return FP4ATTN_OK;
-    if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out) || ((uintptr_t)scales & 7))
+    if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out) ||
+        ((uintptr_t)scales & (uintptr_t)(s.D / 16 - 1)))  // a row's scales: 8 bytes (4 for 64 channels)
         return FP4ATTN_ERR_INVALID_ARG;
-    return launch_status(launch_dequant(codes, scales, g, heads(s) * s.N, out, stream));
+    return launch_status(launch_dequant(codes, scales, g, heads(s) * s.N * (s.D / 16), out, stream));
 }
 
 int fp4attn_read_status(const void* workspace, cudaStream_t stream, int* device_status) {

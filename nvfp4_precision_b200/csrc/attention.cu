@@ -120,8 +120,10 @@ struct __align__(1024) FwdSmem {
 };
 
 struct FwdParams {
-    const uint64_t* q_scales;  // one uint64 (8 UE4M3 bytes) per row
-    const uint64_t* k_scales;
+    const uint8_t* q_scales;  // srb UE4M3 bytes per row
+    const uint8_t* k_scales;
+    int srb;                  // scale bytes per row: 8 (128 channels) or 4 (64)
+    int o_chunks;             // 32-channel chunks of O to store: 4, or 2 for 64 channels
     int N;
     int n_kt;          // K/V stages of BN keys
     float scale_log2;  // softmax_scale * log2(e)
@@ -261,14 +263,17 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         // issues the bulk tensor copies after the atoms are written.  A query
         // tile that lies past N is copied all the same (the copy fills zeros)
         // and its rows are never stored.
-        const uint64_t* qs_head = p.q_scales + (size_t)bh * N;
-        const uint64_t* ks_head = p.k_scales + (size_t)bh * N;
+        const int srb = p.srb;
+        const uint8_t* qs_head = p.q_scales + (size_t)bh * N * srb;
+        const uint8_t* ks_head = p.k_scales + (size_t)bh * N * srb;
         const int v_b = bh / p.H, v_h = bh - v_b * p.H;  // V is addressed as [B][H][N][128]
         const uint32_t qf = smem_u32(&sm.bar_q_full);
 #pragma unroll
         for (int i = 0; i < QT; ++i) {
             const int r0 = q0 + BM * i;
-            load_scale_atoms(qs_head + (r0 < N ? r0 : 0), N - r0, sm.qs_atom[i][0], sm.qs_atom[i][1], lane);
+            uint64_t w[4];
+            fetch_scales_rows(qs_head + (size_t)(r0 < N ? r0 : 0) * srb, srb, N - r0, lane, w);
+            store_scale_atoms(w, sm.qs_atom[i][0], sm.qs_atom[i][1], lane);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
         int issued = 0;
         uint64_t ksc[4];  // the next stage's scales, fetched before its buffer is free
-        fetch_scales(ks_head, N < BN ? N : BN, lane, ksc);
+        fetch_scales_rows(ks_head, srb, N < BN ? N : BN, lane, ksc);
         for (int j = 0; j < T; ++j) {
             const int s = j % STAGES;
             if (j >= STAGES) {
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             store_scale_atoms(ksc, sm.ks_atom[s][0], sm.ks_atom[s][1], lane);
             if (j + 1 < T) {
                 const int rest = N - k0 - BN;
-                fetch_scales(ks_head + k0 + BN, rest < BN ? rest : BN, lane, ksc);
+                fetch_scales_rows(ks_head + (size_t)(k0 + BN) * srb, srb, rest < BN ? rest : BN, lane, ksc);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -553,10 +558,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
             __nv_bfloat16* o_row = p.o + ob * p.o_sb + oh * p.o_sh + (long long)n * p.o_sn;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
+                if (q >= p.o_chunks) break;  // warp-uniform
                 uint32_t r[32];
                 tmem_ld32(o_addr + 32u * q, r);
                 tmem_wait_ld();
-                if (n < N) {
+                if (n < N && FP4ATTN_IN_BOUNDS(bh < (int)gridDim.y, p.status)) {
                     uint4* dst = reinterpret_cast<uint4*>(o_row + 32 * q);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
@@ -570,7 +576,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                     }
                 }
             }
-            if (p.lse && n < N) p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
+            if (p.lse && n < N && FP4ATTN_IN_BOUNDS(orow < (size_t)gridDim.y * N, p.status))
+                p.lse[orow] = (m_run + __log2f(l)) * 0.69314718055994530942f;
         }
     }
 
@@ -722,11 +729,13 @@ struct Maps {
     CUtensorMap qc, kc, v;
 };
 
-// V [B][H][N][128 bf16] with element strides st (multiples of 8): 128B-swizzled
+// V [B][H][N][d bf16] with element strides st (multiples of 8): 128B-swizzled
 // boxes of 64 channels x box_rows keys of one head; x is 0 or 64 (0 or 128
 // bytes), so every box starts on a 16-byte boundary.
-bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, Strides st, uint32_t box_rows) {
-    const uint64_t dims[4] = {128, (uint64_t)N, (uint64_t)H, (uint64_t)B};
+bool make_v_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int N, Strides st, uint32_t box_rows,
+                int d = 128) {
+    // with d = 64 the box of channels 64-127 lies past the row: it reads zeros
+    const uint64_t dims[4] = {(uint64_t)d, (uint64_t)N, (uint64_t)H, (uint64_t)B};
     const uint64_t strides[3] = {(uint64_t)st.n * 2, (uint64_t)st.h * 2, (uint64_t)st.b * 2};
     const uint32_t box[4] = {64, box_rows, 1, 1};
     return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(base),
@@ -741,8 +750,10 @@ size_t probe_smem_bytes() { return sizeof(ProbeSmem) + 1024; }
 int launch_forward(const FwdArgs& a, cudaStream_t stream) {
     if (a.BH == 0 || a.N == 0) return FP4ATTN_OK;
     Maps m;
-    if (!make_code_map(&m.qc, a.q_codes, a.BH, a.N, BM) || !make_code_map(&m.kc, a.k_codes, a.BH, a.N, BN) ||
-        !make_v_map(&m.v, a.v, a.BH / a.H, a.H, a.N, a.vs, BN))
+    const uint32_t code_bytes = (uint32_t)a.d / 2;
+    if (!make_code_map(&m.qc, a.q_codes, a.BH, a.N, BM, code_bytes) ||
+        !make_code_map(&m.kc, a.k_codes, a.BH, a.N, BN, code_bytes) ||
+        !make_v_map(&m.v, a.v, a.BH / a.H, a.H, a.N, a.vs, BN, a.d))
         return FP4ATTN_ERR_CUDA;
     static_assert(sizeof(FwdSmem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = fwd_smem_bytes();
@@ -750,11 +761,14 @@ int launch_forward(const FwdArgs& a, cudaStream_t stream) {
         cudaSuccess)
         return FP4ATTN_ERR_CUDA;
     FwdParams p;
-    p.q_scales = reinterpret_cast<const uint64_t*>(a.q_scales);
-    p.k_scales = reinterpret_cast<const uint64_t*>(a.k_scales);
+    p.q_scales = a.q_scales;
+    p.k_scales = a.k_scales;
+    p.srb = a.d / 16;
+    p.o_chunks = a.d / 32;
     p.N = a.N;
     p.n_kt = (a.N + BN - 1) / BN;
-    const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 0.08838834764831845f;
+    const float scale = a.softmax_scale > 0.0f ? a.softmax_scale
+                                               : (a.d == 64 ? 0.125f : 0.08838834764831845f);  // 1/sqrt(d)
     p.scale_log2 = scale * 1.4426950408889634f;
     p.gq = a.gq;
     p.gk = a.gk;

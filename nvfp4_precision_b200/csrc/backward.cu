@@ -891,8 +891,8 @@ int launch_backward(const BwdArgs& a, cudaStream_t stream) {
     const int B = a.BH / a.H;
     // unit-scale Q~, K~ in bf16 (exact) for the dK / dV kernel and the dQ^ product
     const int64_t rows = (int64_t)a.BH * a.N;
-    if (launch_dequant_bf16(a.q_codes, a.q_scales, nullptr, rows, a.qhat, stream) != cudaSuccess ||
-        launch_dequant_bf16(a.k_codes, a.k_scales, nullptr, rows, a.khat, stream) != cudaSuccess)
+    if (launch_dequant_bf16(a.q_codes, a.q_scales, nullptr, rows * 8, a.qhat, stream) != cudaSuccess ||
+        launch_dequant_bf16(a.k_codes, a.k_scales, nullptr, rows * 8, a.khat, stream) != cudaSuccess)
         return FP4ATTN_ERR_CUDA;
     CUtensorMap qc_r, kc_s, kc_r, qc_s, do_r, k_s, v_s, v_r, q_s, do_s;
     const Strides cs = contiguous_strides(a.H, a.N);  // Q~, K~: the library's own contiguous tensors

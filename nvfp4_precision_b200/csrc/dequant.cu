@@ -78,9 +78,8 @@ cudaError_t launch_div6_check(unsigned* res, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t nblocks,
                            float* out, cudaStream_t stream) {
-    const int64_t nblocks = rows * 8;
     if (nblocks == 0) return cudaSuccess;
     const int threads = 256;
     dequant_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, stream>>>(
@@ -88,9 +87,8 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const fl
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+cudaError_t launch_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t nblocks,
                                 __nv_bfloat16* out, cudaStream_t stream) {
-    const int64_t nblocks = rows * 8;
     if (nblocks == 0) return cudaSuccess;
     const int threads = 256;
     dequant_bf16_kernel<<<(unsigned)((nblocks + threads - 1) / threads), threads, 0, stream>>>(codes, scales, g,

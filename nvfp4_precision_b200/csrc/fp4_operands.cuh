@@ -32,6 +32,23 @@ __device__ __forceinline__ void fetch_scales(const uint64_t* rows, int n_rows, i
     }
 }
 
+// The same for rows of srb = 8 or 4 scale bytes (128 or 64 channels): a row of
+// 4 bytes reads as its 8-byte form with the upper four scales zero.
+__device__ __forceinline__ void fetch_scales_rows(const uint8_t* rows, int srb, int n_rows, int lane,
+                                                  uint64_t (&w)[4]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int r = lane + 32 * c;
+        if (r >= n_rows) {
+            w[c] = 0ull;
+        } else if (srb == 8) {
+            w[c] = __ldg(reinterpret_cast<const unsigned long long*>(rows) + r);
+        } else {
+            w[c] = (uint64_t)__ldg(reinterpret_cast<const unsigned int*>(rows) + r);
+        }
+    }
+}
+
 __device__ __forceinline__ void store_scale_atoms(const uint64_t (&w)[4], uint8_t* atom0, uint8_t* atom1, int lane) {
     *reinterpret_cast<uint4*>(atom0 + 16 * lane) =
         make_uint4((uint32_t)w[0], (uint32_t)w[1], (uint32_t)w[2], (uint32_t)w[3]);
@@ -57,10 +74,13 @@ __device__ __forceinline__ uint64_t codes_desc(const uint8_t* tile, int kchunk) 
     return smem_desc(smem_u32(tile) + 32u * kchunk, 16, 512, LAYOUT_SW64);
 }
 
-// Codes [BH][N][64 bytes]: 64B-swizzled boxes of box_rows rows; x is always 0.
-inline bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N, uint32_t box_rows) {
-    const uint64_t dims[3] = {64, (uint64_t)N, (uint64_t)BH};
-    const uint64_t strides[2] = {64, (uint64_t)N * 64};
+// Codes [BH][N][row_bytes] (64 bytes for 128 channels, 32 for 64): 64B-swizzled
+// boxes of 64 bytes x box_rows rows, x always 0; bytes of a box past a 32-byte
+// row read as zero codes.
+inline bool make_code_map(CUtensorMap* m, const uint8_t* base, int BH, int N, uint32_t box_rows,
+                          uint32_t row_bytes = 64) {
+    const uint64_t dims[3] = {row_bytes, (uint64_t)N, (uint64_t)BH};
+    const uint64_t strides[2] = {row_bytes, (uint64_t)N * row_bytes};
     const uint32_t box[3] = {64, box_rows, 1};
     return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims,
                              strides, box, CU_TENSOR_MAP_SWIZZLE_64B);

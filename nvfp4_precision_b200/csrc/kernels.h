@@ -9,6 +9,18 @@ namespace fp4attn {
 
 constexpr int D = 128;
 
+// Bounds-checked build (-DFP4ATTN_BOUNDS_CHECK): the kernels test each global
+// store, atomic and tile coordinate against the sizes of their buffers; a
+// failed test records FP4ATTN_ERR_RANGE in the status word and skips the
+// access instead of touching memory it does not own.  Without the macro
+// every check is the constant true and compiles away.
+#ifdef FP4ATTN_BOUNDS_CHECK
+#define FP4ATTN_IN_BOUNDS(cond, status)                                                   \
+    ((cond) ? true : (((status) ? (void)atomicCAS((status), 0, (int)FP4ATTN_ERR_RANGE) : (void)0), false))
+#else
+#define FP4ATTN_IN_BOUNDS(cond, status) true
+#endif
+
 // Workspace layout: [0,4) status word, [64,68) and [68,72) tile ticket
 // counters of the two prologue launches, [128,136) fp32 bit patterns of the
 // transformed amax of Q and K (dynamic global scales), rest of [0,256) spare;
@@ -28,8 +40,8 @@ inline size_t ws_bytes(int64_t BH) {
 struct Strides {
     int64_t b, h, n;
 };
-inline Strides contiguous_strides(int H, int N) {
-    return Strides{(int64_t)H * N * D, (int64_t)N * D, (int64_t)D};
+inline Strides contiguous_strides(int H, int N, int d = D) {
+    return Strides{(int64_t)H * N * d, (int64_t)N * d, (int64_t)d};
 }
 
 // Flag of QuantArgs: compute g of Q and K from the transformed amax.
@@ -57,12 +69,33 @@ struct QuantArgs {
 };
 
 cudaError_t launch_quantize_qk(const QuantArgs& a, cudaStream_t stream);
+
+// Heads of 64 channels (codes [B,H,N,32], scales [B,H,N,4], key mean [B,H,64]);
+// static global scales only.  The key sums use the first 64 slots of each
+// head's 128 in the workspace.
+struct Prologue64Args {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    Strides qs, ks;
+    int BH, H, N;
+    uint32_t flags;
+    const float* gq;
+    const float* gk;
+    uint8_t* q_codes;
+    uint8_t* q_scales;
+    uint8_t* k_codes;
+    uint8_t* k_scales;
+    float* k_mean;
+    long long* ksum;
+    int* status;
+};
+cudaError_t launch_quantize_qk64(const Prologue64Args& a, cudaStream_t stream);
 // Test hook: the prologue with its key-sum tiles withheld (K tiles time out).
 cudaError_t launch_quantize_qk_withheld_sums(const QuantArgs& a, uint64_t spin_limit_ns, cudaStream_t stream);
 // Dynamic global scales of empty tensors (amax 0): store the smallest g, 2^-64.
 cudaError_t launch_store_gscales(float* gq, float* gk, cudaStream_t stream);
 
-cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t nblocks,
                            float* out, cudaStream_t stream);
 cudaError_t launch_div6_check(unsigned* res, cudaStream_t stream);
 cudaError_t launch_encode_f32(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
@@ -84,6 +117,7 @@ struct FwdArgs {
     const __nv_bfloat16* v;
     Strides vs, os;
     int BH, H, N;
+    int d;  // 128, or 64: codes [.., 32], scales [.., 4], V and O [.., 64]
     float softmax_scale;
     __nv_bfloat16* o;
     float* lse;
@@ -148,7 +182,7 @@ struct BwdArgs {
 
 // Returns 0 on success, else an fp4attn_status code.
 int launch_backward(const BwdArgs& a, cudaStream_t stream);
-cudaError_t launch_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t rows,
+cudaError_t launch_dequant_bf16(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t nblocks,
                                 __nv_bfloat16* out, cudaStream_t stream);
 int launch_forward(const FwdArgs& a, cudaStream_t stream);
 int launch_forward_bf16qk(const FwdBf16Args& a, cudaStream_t stream);

@@ -313,15 +313,9 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
                     if (run < total) run_next = (int)atomicAdd(a.ticket, (unsigned)run_len);
                 }
                 const int t = run + in_run++;
-#ifdef FP4ATTN_PRO_SPIN
-                if (i >= NSLOT &&
-                    !mbar_wait_spin(smem_u32(&sm.empty[s]), ph ^ 1u, &sm.abort_flag, a.status, kWaitLimitNs))
-                    break;
-#else
                 if (i >= NSLOT &&
                     !mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, &sm.abort_flag, a.status, kWaitLimitNs))
                     break;
-#endif
                 const uint32_t fb = smem_u32(&sm.full[s]);
                 filled |= 1u << s;
                 parity = (parity & ~(1u << s)) | (ph << s);
@@ -332,6 +326,10 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
                 }
                 int kind, bh, tile;
                 decode_ticket(t, Th, a.BH, sums, a.lead, kind, bh, tile);
+                if (!FP4ATTN_IN_BOUNDS(bh >= 0 && bh < a.BH && tile >= 0 && tile < Th && kind <= KIND_K, a.status)) {
+                    sm.abort_flag = 1;
+                    break;
+                }
                 sm.meta[s] = make_int4(kind, bh, tile, 0);
                 const CUtensorMap* map = (kind == KIND_Q) ? &tm_q : &tm_k;
                 const uint64_t pol = (kind == KIND_KSUM) ? pol_keep : pol_stream;
@@ -412,7 +410,7 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             __threadfence_block();
             last = (atomicAdd(&sm.run_warps[b], 1) == W - 1);
         }
-        if (__shfl_sync(0xffffffffu, last, 0)) {
+        if (__shfl_sync(0xffffffffu, last, 0) && FP4ATTN_IN_BOUNDS(pend_bh >= 0 && pend_bh < a.BH, a.status)) {
             __threadfence_block();
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -440,11 +438,7 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
         const uint32_t ph = (uint32_t)(i / NSLOT) & 1u;
         const uint32_t fb = smem_u32(&sm.full[s]);
         {
-#ifdef FP4ATTN_PRO_SPIN
-            const bool ok = mbar_wait_spin(fb, ph, &sm.abort_flag, a.status, kWaitLimitNs);
-#else
             const bool ok = mbar_wait(fb, ph, &sm.abort_flag, a.status, kWaitLimitNs);
-#endif
             if (!__all_sync(0xffffffffu, ok)) break;
         }
         const int4 mt = sm.meta[s];
@@ -646,7 +640,7 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             }
             const uint32_t mine = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
             const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-            if (valid) {
+            if (valid && FP4ATTN_IN_BOUNDS(row < (size_t)a.BH * N, a.status)) {
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
                     *reinterpret_cast<uint2*>(crow + 8 * blk[g]) = make_uint2(wx[g][0], wx[g][1]);

@@ -14,7 +14,11 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfp4attn.so")
+# FP4ATTN_BOUNDS_CHECK=1 selects the bounds-checked build of the same library
+# (build.py --checked): every kernel checks its global stores, atomics and tile
+# coordinates and reports FP4ATTN_ERR_RANGE instead of an out-of-range access.
+LIB_PATH = os.path.join(_PKG, "libfp4attn_checked.so" if os.environ.get("FP4ATTN_BOUNDS_CHECK") == "1"
+                        else "libfp4attn.so")
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -171,11 +175,11 @@ def fp4attn_quantize_qk(q: torch.Tensor, k: torch.Tensor, q_gscale: Optional[tor
     B, H, N, D = q.shape
     dev = q.device
     if out is None:
-        out = dict(q_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
-                   q_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
-                   k_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
-                   k_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
-                   k_mean=torch.empty((B, H, 128), dtype=torch.float32, device=dev) if k_mean else None)
+        out = dict(q_codes=torch.empty((B, H, N, D // 2), dtype=torch.uint8, device=dev),
+                   q_scales=torch.empty((B, H, N, D // 16), dtype=torch.uint8, device=dev),
+                   k_codes=torch.empty((B, H, N, D // 2), dtype=torch.uint8, device=dev),
+                   k_scales=torch.empty((B, H, N, D // 16), dtype=torch.uint8, device=dev),
+                   k_mean=torch.empty((B, H, D), dtype=torch.float32, device=dev) if k_mean else None)
     if workspace is None:
         workspace = new_workspace(B, H, N, dev)
     if dynamic_gscale:
@@ -206,11 +210,11 @@ def fp4attn_quantize_qk_noalloc(q: torch.Tensor, k: torch.Tensor, q_gscale: Opti
     B, H, N, D = q.shape
     dev = q.device
     if out is None:
-        out = dict(q_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
-                   q_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
-                   k_codes=torch.empty((B, H, N, 64), dtype=torch.uint8, device=dev),
-                   k_scales=torch.empty((B, H, N, 8), dtype=torch.uint8, device=dev),
-                   k_mean=torch.empty((B, H, 128), dtype=torch.float32, device=dev) if k_mean else None)
+        out = dict(q_codes=torch.empty((B, H, N, D // 2), dtype=torch.uint8, device=dev),
+                   q_scales=torch.empty((B, H, N, D // 16), dtype=torch.uint8, device=dev),
+                   k_codes=torch.empty((B, H, N, D // 2), dtype=torch.uint8, device=dev),
+                   k_scales=torch.empty((B, H, N, D // 16), dtype=torch.uint8, device=dev),
+                   k_mean=torch.empty((B, H, D), dtype=torch.float32, device=dev) if k_mean else None)
     rc = lib.fp4attn_quantize_qk_noalloc(_ptr(q), _ptr(k), Shape(B, H, N, D), _ptr(q_gscale), _ptr(k_gscale),
                                          int(flags), _ptr(out["q_codes"]), _ptr(out["q_scales"]),
                                          _ptr(out["k_codes"]), _ptr(out["k_scales"]), _ptr(out.get("k_mean")),
@@ -270,9 +274,9 @@ def fp4attn_forward_bf16qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, so
 
 def fp4attn_dequant(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[torch.Tensor] = None,
                     stream=None) -> torch.Tensor:
-    B, H, N, _ = codes.shape
-    out = torch.empty((B, H, N, 128), dtype=torch.float32, device=codes.device)
-    rc = lib.fp4attn_dequant(_ptr(codes), _ptr(scales), _ptr(gscale), Shape(B, H, N, 128), _ptr(out),
+    B, H, N, C = codes.shape  # C = D / 2 code bytes per row
+    out = torch.empty((B, H, N, 2 * C), dtype=torch.float32, device=codes.device)
+    rc = lib.fp4attn_dequant(_ptr(codes), _ptr(scales), _ptr(gscale), Shape(B, H, N, 2 * C), _ptr(out),
                              _stream(stream))
     _check(rc, "fp4attn_dequant")
     return out
@@ -280,10 +284,10 @@ def fp4attn_dequant(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[
 
 def fp4attn_dequant_bf16(codes: torch.Tensor, scales: torch.Tensor, gscale: Optional[torch.Tensor] = None,
                          stream=None) -> torch.Tensor:
-    """NVFP4 [B,H,N,64] codes + [B,H,N,8] scales -> bf16 [B,H,N,128] values."""
-    B, H, N, _ = codes.shape
-    out = torch.empty((B, H, N, 128), dtype=torch.bfloat16, device=codes.device)
-    rc = lib.fp4attn_dequant_bf16(_ptr(codes), _ptr(scales), _ptr(gscale), Shape(B, H, N, 128), _ptr(out),
+    """NVFP4 [B,H,N,D/2] codes + [B,H,N,D/16] scales -> bf16 [B,H,N,D] values."""
+    B, H, N, C = codes.shape
+    out = torch.empty((B, H, N, 2 * C), dtype=torch.bfloat16, device=codes.device)
+    rc = lib.fp4attn_dequant_bf16(_ptr(codes), _ptr(scales), _ptr(gscale), Shape(B, H, N, 2 * C), _ptr(out),
                                   _stream(stream))
     _check(rc, "fp4attn_dequant_bf16")
     return out

@@ -19,7 +19,7 @@ power-of-two width in numpy, with the same pinned steps as the C oracle:
     as the first d/16 blocks of the C pack of the zero-padded 128-wide row.
 Attention is fp64 over the dequantised Q and K, with the exponentials of each
 row (row max subtracted) rounded to bf16 for P.V and the row sum taken over
-the unrounded ones, as in the kernel."""
+those rounded values, as in the kernel (P and V stay in BF16)."""
 from __future__ import annotations
 
 import numpy as np
@@ -54,43 +54,61 @@ def _pad128(x: np.ndarray) -> np.ndarray:
     return out
 
 
-def prologue(q_bits: np.ndarray, k_bits: np.ndarray, flags: int = 0):
-    """Smooth K, rotate, NVFP4-pack and dequantise one set of heads of width
-    d (multiple of 16, at most 128, a power of two when rotating).  q_bits,
-    k_bits: uint16 bf16 bits [H, N, d].  Returns (qhat, khat) float32
-    [H, N, d] (unit global scale: exact values of scale x E2M1)."""
+def quantize(q_bits: np.ndarray, k_bits: np.ndarray, flags: int = 0) -> dict:
+    """Smooth K, rotate and NVFP4-pack one set of heads of width d (multiple
+    of 16, at most 128, a power of two when rotating) at unit global scale.
+    q_bits, k_bits: uint16 bf16 bits [H, N, d].  Returns dict(q_codes,
+    k_codes [H, N, d/2] uint8 (element 2i in the low nibble of byte i),
+    q_scales, k_scales [H, N, d/16] uint8 (UE4M3), k_mean [H, d] float32)."""
     H, N, d = q_bits.shape
     assert d % 16 == 0 and d <= 128
     q = _bits_to_f32(q_bits)
     k = _bits_to_f32(k_bits)
+    mean = np.zeros((H, d), np.float32)
     if not flags & NO_SMOOTH_K:
         S, st = ksum(_pad128(np.ascontiguousarray(k_bits, dtype=np.uint16)))
         assert st == 0
-        k = k - kmean(S, N)[:, None, :d]
+        mean = kmean(S, N)[:, :d]
+        k = k - mean[:, None, :]
     if not flags & NO_HADAMARD:
         c = np.float32(1.0 / np.sqrt(float(d)))
         q = fwht(q) * c
         k = fwht(k) * c
-    out = []
-    for y in (q, k):
+    out = dict(k_mean=mean)
+    for name, y in (("q", q), ("k", k)):
         codes, scales = quantize_rows(_pad128(y.reshape(-1, d)))
-        out.append(dequant(codes, scales)[:, :d].reshape(H, N, d))
+        out[name + "_codes"] = codes[:, : d // 2].reshape(H, N, d // 2)
+        out[name + "_scales"] = scales[:, : d // 16].reshape(H, N, d // 16)
+    return out
+
+
+def prologue(q_bits: np.ndarray, k_bits: np.ndarray, flags: int = 0):
+    """quantize() followed by dequantisation: returns (qhat, khat) float32
+    [H, N, d] (unit global scale: exact values of scale x E2M1)."""
+    c = quantize(q_bits, k_bits, flags)
+    d = q_bits.shape[-1]
+    out = []
+    for t in ("q", "k"):
+        codes = np.zeros(c[t + "_codes"].shape[:-1] + (64,), np.uint8)
+        scales = np.zeros(c[t + "_scales"].shape[:-1] + (8,), np.uint8)
+        codes[..., : d // 2] = c[t + "_codes"]
+        scales[..., : d // 16] = c[t + "_scales"]
+        out.append(dequant(codes, scales)[..., :d])
     return out[0], out[1]
 
 
 def attention(qhat: np.ndarray, khat: np.ndarray, v_bits: np.ndarray, bf16_p: bool = True) -> np.ndarray:
     """fp64 softmax(Q K^T / sqrt(d)) V of each head [H, N, d]; with bf16_p the
-    row's exponentials are rounded to bf16 before P.V (the row sum uses them
-    unrounded)."""
+    row's exponentials are rounded to bf16 before P.V and the row sum is taken
+    over the rounded values."""
     q = np.asarray(qhat, dtype=np.float64)
     k = np.asarray(khat, dtype=np.float64)
     v = _bits_to_f32(v_bits).astype(np.float64)
     s = q @ np.swapaxes(k, -1, -2) / np.sqrt(float(q.shape[-1]))
     p = np.exp(s - s.max(axis=-1, keepdims=True))
-    l = p.sum(axis=-1, keepdims=True)
     if bf16_p:
         p = _round_bf16(p)
-    return (p @ v) / l
+    return (p @ v) / p.sum(axis=-1, keepdims=True)
 
 
 def _round_bf16(x: np.ndarray) -> np.ndarray:

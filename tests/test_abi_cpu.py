@@ -52,7 +52,13 @@ def _q(fa, shape, ws=ctypes.c_void_p(256), wsb=1 << 20, flags=0, ptr=ctypes.c_vo
 
 def test_quantize_validation_before_launch(fa):
     S = fa.Shape
-    assert _q(fa, S(1, 1, 128, 64)) == fa.ERR_UNSUPPORTED          # D != 128
+    assert _q(fa, S(1, 1, 128, 96)) == fa.ERR_UNSUPPORTED          # D other than 64 or 128
+    assert _q(fa, S(1, 1, 128, 256)) == fa.ERR_UNSUPPORTED
+    assert fa.lib.fp4attn_quantize_qk_ex(ctypes.c_void_p(4096), fa.Strides(0, 0, 0), ctypes.c_void_p(4096),
+                                         fa.Strides(0, 0, 0), S(1, 1, 128, 64), ctypes.c_void_p(4096),
+                                         ctypes.c_void_p(4096), fa.DYNAMIC_GSCALE, *(4 * [ctypes.c_void_p(4096)]),
+                                         None, ctypes.c_void_p(256), 1 << 20, None) \
+        == fa.ERR_UNSUPPORTED                                       # dynamic scales: 128 channels only
     assert _q(fa, S(1, -1, 128, 128)) == fa.ERR_INVALID_ARG        # negative size
     assert _q(fa, S(1, 1, 1 << 19, 128)) == fa.ERR_UNSUPPORTED     # N beyond the exact-sum range
     assert _q(fa, S(1, 1, (1 << 18) + 1, 128)) == fa.ERR_UNSUPPORTED
@@ -68,6 +74,9 @@ def test_forward_validation_before_launch(fa):
     p = ctypes.c_void_p(4096)
     f = fa.lib.fp4attn_forward
     assert f(p, p, p, p, None, None, p, S(1, 1, 128, 96), 0.0, p, None, p, 1 << 20, None) == fa.ERR_UNSUPPORTED
+    # the BF16-QK attention and the training backward take 128 channels only
+    assert fa.lib.fp4attn_forward_bf16qk(p, p, p, S(1, 1, 128, 64), 0.0, p, None, p, 1 << 20, None) \
+        == fa.ERR_UNSUPPORTED
     assert f(p, p, p, p, None, None, p, S(1, 1, 128, 128), 0.0, p, None, None, 0, None) == fa.ERR_WORKSPACE
     assert f(None, p, p, p, None, None, p, S(1, 1, 128, 128), 0.0, p, None, p, 1 << 20, None) == fa.ERR_INVALID_ARG
     assert f(p, p, p, p, None, None, p, S(1, 1, 128, 128), float("nan"), p, None, p, 1 << 20, None) \
