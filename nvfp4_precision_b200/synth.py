@@ -63,9 +63,9 @@ class Workload:
                 f" tail={self.tail_rows}@{self.tail_std} seed={self.seed}")
 
 
-# The five workloads: tiny correctness, mid, 5-second clip (with a ~1k audio
-# tail), 15-second clip (the 109k-token headline), and the heavy-tailed
-# quantisation-prologue stress case.
+# The workloads: tiny correctness, mid, 5-second clip (with a ~1k audio
+# tail), 15-second clip (the 109k-token headline), eight heads of it, and the
+# heavy-tailed quantisation-prologue stress case.
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 2, 512, seed=0, k_offset_std=2.0),
     "mid": Workload("mid", 1, 8, 8192, seed=1, n_outliers=2, outlier_factor=20.0, k_offset_std=2.0),
@@ -73,6 +73,11 @@ WORKLOADS = {
                        k_offset_std=2.0, tail_rows=1024, tail_std=0.5),
     "clip15s": Workload("clip15s", 1, 48, 109568, seed=3, n_outliers=2, outlier_factor=20.0,
                         k_offset_std=2.0),
+    # the 15-second clip's recipe and head length with eight heads: the
+    # headline's per-head access pattern in a few GB of device memory, for
+    # hardware-counter captures of one launch
+    "clip15s_8heads": Workload("clip15s_8heads", 1, 8, 109568, seed=3, n_outliers=2, outlier_factor=20.0,
+                               k_offset_std=2.0),
     "prologue_stress": Workload("prologue_stress", 1, 48, 109568, seed=4, dist="student_t3",
                                 n_outliers=4, outlier_factor=50.0, with_v=False),
 }
