@@ -11,10 +11,11 @@
 // tickets, one atomic per run) in which every head contributes three runs:
 // key-sum tiles (exact int64 fixed-point column sums of K, the sum of
 // round_half_even(k * 2^24), order-independent), Q tiles and K tiles.  The
-// key sums of head h+1 are placed between the Q and the K tiles of head h,
-// so a K tile rarely waits for its head's sums, while K is still in L2 for
-// its second read (key-sum loads are marked evict-last, the others
-// evict-first).
+// key sums of head h+L are placed between the Q and the K tiles of head h,
+// with the lead L the smallest that keeps every CTA's unfinished tickets
+// from reaching a head's K tiles before its sums are complete, so a K tile
+// does not wait, while K is still in L2 for its second read (key-sum loads
+// are marked evict-last, the others evict-first).
 //
 // Warp W of each CTA is the producer: it takes tickets and moves each tile by
 // TMA (two 128B-swizzled boxes of 64 channels) into a ring of NSLOT shared-
@@ -70,7 +71,7 @@
 #define FP4ATTN_PRO_RUN 8      // most consecutive tiles per ticket request
 #endif
 #ifndef FP4ATTN_PRO_LEAD
-#define FP4ATTN_PRO_LEAD 1     // key sums of head h+1 between Q(h) and K(h)
+#define FP4ATTN_PRO_LEAD 1     // least lead of the key sums over the K tiles (0: ahead of Q(h))
 #endif
 
 namespace fp4attn {
@@ -121,7 +122,7 @@ struct ProArgs {
     uint32_t flags;
     bool sums_ready;   // the key sums of every head are complete: no key-sum tiles
     bool withhold_sums;  // test hook: K tiles wait for key sums that no tile computes
-    int lead;          // 1: key sums of head h+1 between Q(h) and K(h); 0: ahead of Q(h)
+    int lead;          // L >= 1: key sums of head h+L between Q(h) and K(h); 0: ahead of Q(h)
     int run;           // consecutive tiles per ticket request
     uint64_t spin_limit_ns;
     int* status;
@@ -178,9 +179,10 @@ __device__ __forceinline__ void block_scale(float a, float g, bool g_is_one, con
     }
 }
 
-// Ticket t -> (kind, flat head, tile).  With key sums (sums_per_head), head h
-// contributes [Q(h)][key sums of h+1][K(h)] after a first run of the key sums
-// of head 0 (lead 1), or [key sums of h][Q(h)][K(h)] (lead 0).
+// Ticket t -> (kind, flat head, tile).  With key sums (sums), lead L >= 1:
+// the key sums of heads 0..L-1 first, then per head h [Q(h)][key sums of
+// h+L][K(h)] (the last L heads without the middle run); lead 0:
+// [key sums of h][Q(h)][K(h)].
 __device__ __forceinline__ void decode_ticket(int t, int Th, int BH, bool sums, int lead, int& kind, int& bh,
                                               int& tile) {
     if (!sums) {
@@ -198,29 +200,37 @@ __device__ __forceinline__ void decode_ticket(int t, int Th, int BH, bool sums, 
         tile = l - part * Th;
         return;
     }
-    if (t < Th) {
+    const int first = lead < BH ? lead : BH;  // heads whose key sums come first
+    if (t < first * Th) {
         kind = KIND_KSUM;
-        bh = 0;
-        tile = t;
+        bh = t / Th;
+        tile = t - bh * Th;
         return;
     }
-    t -= Th;
-    int h = t / (3 * Th);
-    if (h > BH - 1) h = BH - 1;
-    const int l = t - h * 3 * Th;
-    if (l < Th) {
-        kind = KIND_Q;
-        bh = h;
-        tile = l;
-    } else if (h + 1 < BH && l < 2 * Th) {
-        kind = KIND_KSUM;
-        bh = h + 1;
-        tile = l - Th;
-    } else {
-        kind = KIND_K;
-        bh = h;
-        tile = l - (h + 1 < BH ? 2 * Th : Th);
+    t -= first * Th;
+    const int inner = BH - first;  // heads with a run of later key sums inside
+    if (t < inner * 3 * Th) {
+        const int h = t / (3 * Th), l = t - h * 3 * Th;
+        if (l < Th) {
+            kind = KIND_Q;
+            bh = h;
+            tile = l;
+        } else if (l < 2 * Th) {
+            kind = KIND_KSUM;
+            bh = h + lead;
+            tile = l - Th;
+        } else {
+            kind = KIND_K;
+            bh = h;
+            tile = l - 2 * Th;
+        }
+        return;
     }
+    t -= inner * 3 * Th;
+    const int h = inner + t / (2 * Th), l = t - (h - inner) * 2 * Th;
+    kind = l < Th ? KIND_Q : KIND_K;
+    bh = h;
+    tile = l < Th ? l : l - Th;
 }
 
 // AMAX = true: the first launch of the dynamic-scale path (key sums and the
@@ -277,25 +287,29 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             const uint64_t pol_keep = l2_policy_evict_last();
             const uint64_t pol_stream = l2_policy_evict_first();
             uint32_t filled = 0u, parity = 0u;  // per slot: ever filled; parity of its last fill
-            // tickets come in runs of a.run consecutive tiles, the next
-            // run requested as soon as the current one starts, so the
-            // atomic's round trip overlaps the fills instead of preceding each
+            // tickets come in runs of a.run consecutive tiles.  A ticket is
+            // taken only when its slot is free, and the next run is requested
+            // with the last ticket of the current one and read after the next
+            // slot frees, so the atomic's round trip overlaps that wait and a
+            // CTA never holds more than NSLOT + a.run tickets it has not
+            // finished: few enough that a head's key sums are complete before
+            // its K tiles are handed out (the lead is sized from it).
             const int run_len = a.run;
             int run = (int)atomicAdd(a.ticket, (unsigned)run_len);
-            int run_next = (int)atomicAdd(a.ticket, (unsigned)run_len);
+            int run_next = 0;
             int in_run = 0;
             for (int i = 0;; ++i) {
                 const int s = i % NSLOT;
                 const uint32_t ph = (uint32_t)(i / NSLOT) & 1u;
-                if (in_run == run_len) {
-                    run = run_next;
-                    in_run = 0;
-                    if (run < total) run_next = (int)atomicAdd(a.ticket, (unsigned)run_len);
-                }
-                const int t = run + in_run++;
                 if (i >= NSLOT &&
                     !mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, &sm.abort_flag, a.status, kWaitLimitNs))
                     break;
+                if (in_run == run_len) {
+                    run = run_next;
+                    in_run = 0;
+                }
+                const int t = run + in_run++;
+                if (in_run == run_len && t < total) run_next = (int)atomicAdd(a.ticket, (unsigned)run_len);
                 const uint32_t fb = smem_u32(&sm.full[s]);
                 filled |= 1u << s;
                 parity = (parity & ~(1u << s)) | (ph << s);
@@ -673,7 +687,17 @@ cudaError_t launch_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const 
     const long long tiles = (long long)a.BH * a.n_tiles * (sum_tiles ? 3 : 2);
     long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
     if (grid > tiles) grid = tiles;
-    prologue_kernel<AMAX><<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, a);
+    ProArgs b = a;
+    if (sum_tiles && b.lead > 0) {
+        // A head's K tiles are handed out about 3 * lead * n_tiles tickets
+        // after its last key-sum tile, and the CTAs hold at most
+        // grid * (NSLOT + run) tickets they have not finished: the smallest
+        // lead that keeps the first a quarter above the second lets no K tile
+        // wait for its sums, while K is still in L2 for its second read.
+        const long long held = grid * (NSLOT + b.run);
+        while (b.lead < b.BH && 3LL * b.lead * b.n_tiles < held + held / 4) ++b.lead;
+    }
+    prologue_kernel<AMAX><<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, b);
     return cudaGetLastError();
 }
 
@@ -700,10 +724,8 @@ ProArgs base_args(const QuantArgs& q) {
     a.n_tiles = (q.N + TILE_ROWS - 1) / TILE_ROWS;
     a.flags = q.flags & ~QUANT_DYNAMIC_G;
     a.lead = FP4ATTN_PRO_LEAD;
-    // The tiles taken but not yet finished across the GPU (the CTAs' rings plus
-    // two ticket runs each) must stay well below the distance from a head's
-    // key-sum tiles to its K tiles (three runs of n_tiles), or K tiles wait:
-    // runs of about n_tiles / 48 tiles, 1 to MAX_TICKET_RUN.
+    // runs of about n_tiles / 48 tiles, 1 to MAX_TICKET_RUN (the lead, set at
+    // launch, grows with the tickets the CTAs can hold)
     a.run = a.n_tiles / 48;
     if (a.run < 1) a.run = 1;
     if (a.run > MAX_TICKET_RUN) a.run = MAX_TICKET_RUN;
