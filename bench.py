@@ -57,11 +57,12 @@ PAGES_CONTEXT = {
 # length, a few GB on the device) times six: heads are independent and the
 # traffic of a launch grows with their number.
 ATTN_TRAFFIC_BYTES = {
-    ("5e2fc71fa917c49f", "clip15s_8heads"): 0.4428e9 + 0.2073e9,
-    ("5e2fc71fa917c49f", "clip15s"): 6 * (0.4428e9 + 0.2073e9),
+    ("5e2fc71fa917c49f", "clip15s_8heads"): 0.4297e9 + 0.2081e9,
+    ("5e2fc71fa917c49f", "clip15s"): 6 * (0.4297e9 + 0.2081e9),
 }
 PROLOGUE_TRAFFIC_BYTES = {
-    ("2abaa5cb75d16bd1", "clip15s"): 2.703e9 + 0.723e9,
+    ("cc3c0d927130d9c1", "clip15s_8heads"): 0.5991e9 + 0.0748e9,
+    ("cc3c0d927130d9c1", "clip15s"): 6 * (0.5991e9 + 0.0748e9),
 }
 
 
@@ -466,6 +467,20 @@ def run_ours(args, rank, world, local):
                     "launches": 6}
         del dout, bws
 
+    # ---- the tensor-core rates behind the composite roofline (context for
+    # its nominal FP4:BF16 ratio of 4): block-scaled FP4 and BF16 MMAs back to
+    # back on every SM, operands resident, outside the timed step ----
+    rates = None
+    if not args.no_rates:
+        r4 = fa.fp4attn_probe_mma_rate(0, reps=40000, stream=stream)
+        r16 = fa.fp4attn_probe_mma_rate(1, reps=10000, stream=stream)
+        rates = {"fp4_tflops": r4["tflops"], "bf16_tflops": r16["tflops"],
+                 "fp4_flop_per_clk_sm": r4["flop_per_clk_sm"], "bf16_flop_per_clk_sm": r16["flop_per_clk_sm"],
+                 "fp4_to_bf16_per_clock": r4["flop_per_clk_sm"] / r16["flop_per_clk_sm"],
+                 "sm_mhz": [r4["sm_mhz"], r16["sm_mhz"]],
+                 "what": ("tcgen05 kind::mxf4nvf4 M128 N256 K64 and kind::f16 M128 N256 K16, back to back "
+                          "on every SM, operands in shared memory and TMEM")}
+
     csrc = os.path.join(ROOT, "nvfp4_precision_b200", "csrc")
     traffic = ATTN_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "attention.cu")), args.workload))
     pro_traffic = PROLOGUE_TRAFFIC_BYTES.get((source_hash(os.path.join(csrc, "prologue.cu")), args.workload))
@@ -567,6 +582,7 @@ def run_ours(args, rank, world, local):
                                        f"x nominal FP4:BF16 ratio 4"
                                        + (f", scaled to this run's median SM clock {clocks['sm_mhz']} MHz"
                                           if clock_ratio else ", no clock samples: unscaled"))},
+            "tensor_rates": rates,
             "clocks": clocks,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
@@ -590,6 +606,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-bf16qk", action="store_true", help="skip timing the BF16-QK attention")
     ap.add_argument("--no-train", action="store_true", help="skip timing the training-time backward")
+    ap.add_argument("--no-rates", action="store_true", help="skip the tensor-core rate probe")
     ap.add_argument("--no-general", action="store_true",
                     help="skip timing the dynamic-scale prologue and the [B,N,H,128] layout")
     args = ap.parse_args()

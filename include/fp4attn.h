@@ -328,6 +328,21 @@ int fp4attn_probe_pv_tile(const void* p_bf16_dev, const void* v_bf16_dev, float*
  *     smallest mismatching bit pattern (0xFFFFFFFF if none). */
 int fp4attn_probe_div6(uint32_t* result_dev, cudaStream_t stream);
 
+/* Tensor-core rate probe (a measurement of the roofline's denominators, not a
+ * step of the path): one CTA per SM issues `reps` groups of back-to-back
+ * tcgen05 MMAs into one TMEM accumulator, every operand resident.
+ *   mode 0: block-scaled FP4 (kind::mxf4nvf4, scale_vec::4X, E2M1 operands,
+ *           UE4M3 factors per 16 values) M=128 N=256 K=64, two per group:
+ *           2*2*128*256*64 FLOPs per group per SM;
+ *   mode 1: BF16 (kind::f16, fp32 accumulate) M=128 N=256 K=16, eight per
+ *           group: 8*2*128*256*16 FLOPs per group per SM.
+ * *cycles_dev (device int64) receives CTA 0's clock64() count from its first
+ * issue to the completion of its last MMA, or -1 if that completion was not
+ * seen within 4 s (then FP4ATTN_ERR_TIMEOUT is in *status_dev, a device int32
+ * the caller zeroes).  The caller times the launch with events on `stream`.
+ * 1 <= reps <= 10^6; asynchronous. */
+int fp4attn_probe_mma_rate(int mode, int reps, long long* cycles_dev, int* status_dev, cudaStream_t stream);
+
 /* Runs the bounded mbarrier wait of the attention kernel on a barrier that
  * nothing arrives at, with the given limit; the kernel must give up and write
  * FP4ATTN_ERR_TIMEOUT into *status_dev (device int32, set to 0 first). */

@@ -433,6 +433,13 @@ int fp4attn_probe_div6(uint32_t* result, cudaStream_t stream) {
     return launch_status(e);
 }
 
+int fp4attn_probe_mma_rate(int mode, int reps, long long* cycles, int* status, cudaStream_t stream) {
+    if ((mode != 0 && mode != 1) || reps < 1 || reps > 1000000 || !cycles || ((uintptr_t)cycles & 7) || !status ||
+        ((uintptr_t)status & 3))
+        return FP4ATTN_ERR_INVALID_ARG;
+    return launch_status(launch_mma_rate(mode, reps, cycles, status, stream));
+}
+
 int fp4attn_probe_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t stream) {
     if (!status || limit_ns > 10000000000ull) return FP4ATTN_ERR_INVALID_ARG;
     return launch_probe_wait_timeout(status, limit_ns, stream);

@@ -98,6 +98,7 @@ cudaError_t launch_store_gscales(float* gq, float* gk, cudaStream_t stream);
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t nblocks,
                            float* out, cudaStream_t stream);
 cudaError_t launch_div6_check(unsigned* res, cudaStream_t stream);
+cudaError_t launch_mma_rate(int mode, int reps, long long* cycles, int* status, cudaStream_t stream);
 cudaError_t launch_encode_f32(const float* x, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
                               cudaStream_t stream);
 

@@ -38,7 +38,7 @@ EXPORTS = (
     "fp4attn_backward_workspace_bytes",
     "fp4attn_read_status", "fp4attn_reset_status", "fp4attn_status_string", "fp4attn_encode_f32",
     "fp4attn_probe_qk_tile", "fp4attn_probe_pv_tile", "fp4attn_probe_wait_timeout", "fp4attn_probe_div6",
-    "fp4attn_probe_withheld_key_sums",
+    "fp4attn_probe_withheld_key_sums", "fp4attn_probe_mma_rate",
 )
 
 
@@ -107,6 +107,8 @@ def _load():
     L.fp4attn_probe_pv_tile.restype = ctypes.c_int
     L.fp4attn_probe_pv_tile.argtypes = [P, P, P, P]
     L.fp4attn_probe_div6.restype = ctypes.c_int
+    L.fp4attn_probe_mma_rate.restype = ctypes.c_int
+    L.fp4attn_probe_mma_rate.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
     L.fp4attn_probe_div6.argtypes = [P, P]
     L.fp4attn_probe_wait_timeout.restype = ctypes.c_int
     L.fp4attn_probe_wait_timeout.argtypes = [P, U64, P]
@@ -409,6 +411,32 @@ def fp4attn_probe_div6(stream=None):
     _check(lib.fp4attn_probe_div6(_ptr(res), _stream(stream)), "fp4attn_probe_div6")
     r = res.cpu().numpy().view("uint32")
     return int(r[0]), int(r[1])
+
+
+MMA_RATE_FLOPS_PER_GROUP = {0: 2 * 2 * 128 * 256 * 64, 1: 8 * 2 * 128 * 256 * 16}
+
+
+def fp4attn_probe_mma_rate(mode: int, reps: int = 40000, stream=None) -> dict:
+    """Back-to-back tcgen05 MMA throughput on every SM (mode 0: block-scaled
+    FP4 M128 N256 K64; mode 1: BF16 M128 N256 K16), timed by CUDA events on
+    the stream, with the SM clock CTA 0 saw: dict(ms, tflops, flop_per_clk_sm,
+    sm_mhz)."""
+    cycles = torch.zeros(1, dtype=torch.int64, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = stream if stream is not None else torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    _check(lib.fp4attn_probe_mma_rate(mode, reps, _ptr(cycles), _ptr(status), _stream(st)), "fp4attn_probe_mma_rate")
+    e1.record(st)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    cyc = int(cycles.item())
+    if int(status.item()) != 0 or cyc <= 0:
+        raise RuntimeError(f"fp4attn_probe_mma_rate: status {int(status.item())}, cycles {cyc}")
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    flops = MMA_RATE_FLOPS_PER_GROUP[mode] * reps
+    return {"ms": ms, "tflops": flops * sms / (ms * 1e-3) / 1e12, "flop_per_clk_sm": flops / cyc,
+            "sm_mhz": cyc / (ms * 1e3)}
 
 
 def fp4attn_probe_wait_timeout(limit_ns: int, stream=None) -> int:
