@@ -472,6 +472,7 @@ def run_ours(args, rank, world, local):
     # back on every SM, operands resident, outside the timed step ----
     rates = None
     if not args.no_rates:
+        fa.fp4attn_probe_mma_rate(0, reps=4000, stream=stream)  # warm-up
         r4 = fa.fp4attn_probe_mma_rate(0, reps=40000, stream=stream)
         r16 = fa.fp4attn_probe_mma_rate(1, reps=10000, stream=stream)
         rates = {"fp4_tflops": r4["tflops"], "bf16_tflops": r16["tflops"],

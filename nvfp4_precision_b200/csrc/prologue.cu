@@ -165,17 +165,48 @@ __device__ __forceinline__ float amax16(const float2* p, bool hi) {
     return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), 0.0f);
 }
 
-// Scale byte and 1/(g*scale) of one block with amax a.
-__device__ __forceinline__ void block_scale(float a, float g, bool g_is_one, const float* inv_tab, uint32_t& s,
-                                            float& inv) {
-    float t = div6_rn(a);
-    if (!g_is_one) t = __fdiv_rn(t, g);
-    s = cvt_e4m3(t);  // t >= +0: the E4M3 byte is the UE4M3 byte
-    if (g_is_one) {
+// Scale byte and 1/(g*scale) of one 16-value block with amax a >= 0.  The
+// quotient a/6 is fl(a * fl(1/6)) corrected by one FMA: equal to the IEEE
+// quotient for every a >= 2^-123 (checked over all fp32 patterns).  Below
+// that, a/6/g < 2^-61 for every admissible g (g >= 2^-64), far under half of
+// the smallest UE4M3 step (2^-9), so the byte is 0 whatever the low bits of
+// the quotient and no exact-divide path is needed; the sign bit is cleared
+// so that a -0 could not give the byte 0x80.
+template <bool G1>
+__device__ __forceinline__ void block_scale(float a, float g, const float* inv_tab, uint32_t& s, float& inv) {
+    const float r6 = __uint_as_float(0x3E2AAAABu);  // fl(1/6)
+    const float q0 = __fmul_rn(a, r6);
+    float t = __fmaf_rn(__fmaf_rn(-6.0f, q0, a), r6, q0);
+    if (!G1) t = __fdiv_rn(t, g);
+    s = cvt_e4m3(t) & 0x7Fu;
+    if (G1) {
         inv = inv_tab[s];
     } else {
         const float sd = ue4m3_value(s);
         inv = (sd != 0.0f) ? __frcp_rn(__fmul_rn(g, sd)) : 0.0f;
+    }
+}
+
+// NVFP4 pack of a lane's four blocks: group q = P[16q..16q+15], its .x values
+// one block and its .y values another; sb receives the four scale bytes (.x
+// of groups 0, 1, then .y), wx / wy the code words (block order as sb).
+template <bool G1>
+__device__ __forceinline__ void pack_blocks(const float2* P, float g, const float* inv_tab, uint32_t (&sb)[4],
+                                            uint32_t (&wx)[2][2], uint32_t (&wy)[2][2]) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        float inv_x, inv_y;
+        block_scale<G1>(amax16(P + 16 * q, false), g, inv_tab, sb[q], inv_x);
+        block_scale<G1>(amax16(P + 16 * q, true), g, inv_tab, sb[2 + q], inv_y);
+        const float2 inv2 = f2(inv_x, inv_y);
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+            float2 R[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) R[k] = __fmul2_rn(P[16 * q + 8 * h8 + k], inv2);
+            wx[q][h8] = cvt_e2m1x8(R[0].x, R[1].x, R[2].x, R[3].x, R[4].x, R[5].x, R[6].x, R[7].x);
+            wy[q][h8] = cvt_e2m1x8(R[0].y, R[1].y, R[2].y, R[3].y, R[4].y, R[5].y, R[6].y, R[7].y);
+        }
     }
 }
 
@@ -235,7 +266,7 @@ __device__ __forceinline__ void decode_ticket(int t, int Th, int BH, bool sums, 
 
 // AMAX = true: the first launch of the dynamic-scale path (key sums and the
 // transformed amax of Q and K; no codes are written).
-template <bool AMAX>
+template <bool AMAX, bool HAD, bool SMOOTH>
 __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                           const __grid_constant__ CUtensorMap tm_k,
                                                                           const ProArgs a) {
@@ -245,8 +276,8 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
     const int warp = tid >> 5, lane = tid & 31;
     const int N = a.N;
     const int Th = a.n_tiles;
-    const bool smooth = !(a.flags & FP4ATTN_NO_SMOOTH_K);
-    const bool hadamard = !(a.flags & FP4ATTN_NO_HADAMARD);
+    constexpr bool smooth = SMOOTH;  // one instance per setting of the two transforms
+    constexpr bool hadamard = HAD;
     const bool sums = smooth && !a.sums_ready && !a.withhold_sums;
     const int total = a.BH * Th * (sums ? 3 : 2);
 
@@ -612,26 +643,14 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             // its .x values form block blk[g], its .y values block blk[2+g];
             // block b's codes are bytes 8b..8b+7 of the row
             const float gw = which ? gk : gq;
-            const bool g_is_one = (gw == 1.0f);
             const size_t row = (size_t)bh * N + (size_t)tile * TILE_ROWS + r;
             uint8_t* crow = (which ? a.codes[1] : a.codes[0]) + row * 64;
             uint32_t sb[4];
             uint32_t wx[2][2], wy[2][2];
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                float inv_x, inv_y;
-                block_scale(amax16(P + 16 * g, false), gw, g_is_one, sm.inv_scale, sb[g], inv_x);
-                block_scale(amax16(P + 16 * g, true), gw, g_is_one, sm.inv_scale, sb[2 + g], inv_y);
-                const float2 inv2 = f2(inv_x, inv_y);
-#pragma unroll
-                for (int h8 = 0; h8 < 2; ++h8) {
-                    float2 R[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) R[k] = __fmul2_rn(P[16 * g + 8 * h8 + k], inv2);
-                    wx[g][h8] = cvt_e2m1x8(R[0].x, R[1].x, R[2].x, R[3].x, R[4].x, R[5].x, R[6].x, R[7].x);
-                    wy[g][h8] = cvt_e2m1x8(R[0].y, R[1].y, R[2].y, R[3].y, R[4].y, R[5].y, R[6].y, R[7].y);
-                }
-            }
+            if (gw == 1.0f)
+                pack_blocks<true>(P, gw, sm.inv_scale, sb, wx, wy);
+            else
+                pack_blocks<false>(P, gw, sm.inv_scale, sb, wx, wy);
             const uint32_t mine = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
             const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
             if (valid && FP4ATTN_IN_BOUNDS(row < (size_t)a.BH * N, a.status)) {
@@ -671,17 +690,17 @@ bool make_rows_map(CUtensorMap* m, const __nv_bfloat16* base, int B, int H, int 
                              strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <bool AMAX>
-cudaError_t launch_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ProArgs& a, cudaStream_t stream) {
+template <bool AMAX, bool HAD, bool SMOOTH>
+cudaError_t launch_inst(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ProArgs& a, cudaStream_t stream) {
     static_assert(sizeof(ProSmem) + 1024 <= 227 * 1024, "shared memory budget");
     const size_t smem = pro_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(prologue_kernel<AMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const auto kernel = prologue_kernel<AMAX, HAD, SMOOTH>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prologue_kernel<AMAX>, PRO_THREADS, smem)) !=
-        cudaSuccess)
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, PRO_THREADS, smem)) != cudaSuccess)
         return e;
     const bool sum_tiles = !(a.flags & FP4ATTN_NO_SMOOTH_K) && !a.sums_ready && !a.withhold_sums;
     const long long tiles = (long long)a.BH * a.n_tiles * (sum_tiles ? 3 : 2);
@@ -697,8 +716,17 @@ cudaError_t launch_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const 
         const long long held = grid * (NSLOT + b.run);
         while (b.lead < b.BH && 3LL * b.lead * b.n_tiles < held + held / 4) ++b.lead;
     }
-    prologue_kernel<AMAX><<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, b);
+    kernel<<<(unsigned)grid, PRO_THREADS, smem, stream>>>(tm_q, tm_k, b);
     return cudaGetLastError();
+}
+
+template <bool AMAX>
+cudaError_t launch_pass(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ProArgs& a, cudaStream_t stream) {
+    const bool had = !(a.flags & FP4ATTN_NO_HADAMARD), smooth = !(a.flags & FP4ATTN_NO_SMOOTH_K);
+    if (had) return smooth ? launch_inst<AMAX, true, true>(tm_q, tm_k, a, stream)
+                           : launch_inst<AMAX, true, false>(tm_q, tm_k, a, stream);
+    return smooth ? launch_inst<AMAX, false, true>(tm_q, tm_k, a, stream)
+                  : launch_inst<AMAX, false, false>(tm_q, tm_k, a, stream);
 }
 
 __global__ void store_gscales_kernel(float* gq, float* gk) {
