@@ -474,7 +474,6 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
 
         if (kind == KIND_KSUM) {
             // -------------------------------------------------- key sums ----
-            if (pend_cnt && pend_bh != bh && !flush()) break;
             const uint8_t* hb = tb + (lane >> 4) * HALF_BYTES;
             const int j = (lane & 15) >> 1;
             const uint32_t in_chunk = (uint32_t)(lane & 1) * 8u;
@@ -483,6 +482,9 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             for (int rr = 0; rr < 16; ++rr) kw[rr] = *reinterpret_cast<const uint2*>(hb + swz(16 * warp + rr, j) + in_chunk);
             __syncwarp();
             if (lane == 0) mbar_arrive(eb);
+            // a run of another head ends here: flushed after the slot is
+            // released, so the ring refills meanwhile
+            if (pend_cnt && pend_bh != bh && !flush()) break;
             const float2 two24 = f2(kTwo24, kTwo24);
 #pragma unroll
             for (int rr = 0; rr < 16; rr += 2) {
@@ -501,6 +503,22 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             ++pend_cnt;
             continue;
         }
+        // with key sums (a flush or a wait for a head's means may come
+        // next), the row goes into registers and the slot is released first,
+        // so that neither holds a slot; without, the copy comes just before
+        // the arithmetic
+        uint4 rlo[4], rhi[4];
+        auto load_row = [&]() {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int cj = 4 * h + j;
+                rlo[j] = *reinterpret_cast<const uint4*>(tb + swz(r, cj));
+                rhi[j] = *reinterpret_cast<const uint4*>(tb + HALF_BYTES + swz(r, cj));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(eb);
+        };
+        if constexpr (SMOOTH) load_row();
         if (pend_cnt && !flush()) break;
         const int which = kind - 1;  // 0 = Q, 1 = K
         const bool sub_mean = (which == 1) && smooth;
@@ -545,16 +563,8 @@ __global__ void __launch_bounds__(PRO_THREADS, CTAS_PER_SM) prologue_kernel(cons
             mean_head = bh;
         }
         // ------------------------------------------------------- one row ----
-        uint4 rlo[4], rhi[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int cj = 4 * h + j;
-            rlo[j] = *reinterpret_cast<const uint4*>(tb + swz(r, cj));
-            rhi[j] = *reinterpret_cast<const uint4*>(tb + HALF_BYTES + swz(r, cj));
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(eb);
 
+        if constexpr (!SMOOTH) load_row();
         float2 P[32];
         bool finite = true;
         // chunk j (8 pairs): unpack, smooth, and the butterflies of stride
