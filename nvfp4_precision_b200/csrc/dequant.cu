@@ -56,14 +56,18 @@ __global__ void encode_kernel(const float* __restrict__ x, int64_t n, uint8_t* e
     }
 }
 
-// Every non-negative finite fp32 bit pattern: div6_rn against the IEEE quotient.
-// res[0] counts mismatches, res[1] holds the smallest mismatching pattern.
+// Every non-negative finite fp32 bit pattern a: div6_rn(a) against the IEEE
+// quotient, and the UE4M3 byte of the branch-free div6_refined(a) (the block
+// scale at g = 1, sign bit cleared) against the byte of the IEEE quotient.
+// res[0] counts the inputs where either differs, res[1] holds the smallest.
 __global__ void div6_check_kernel(unsigned* res) {
     const uint32_t stride = gridDim.x * blockDim.x;
     unsigned count = 0;
     for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < 0x7F800000u; i += stride) {
         const float a = __uint_as_float(i);
-        if (__float_as_uint(div6_rn(a)) != __float_as_uint(__fdiv_rn(a, 6.0f))) {
+        const float q = __fdiv_rn(a, 6.0f);
+        if (__float_as_uint(div6_rn(a)) != __float_as_uint(q) ||
+            (cvt_e4m3(div6_refined(a)) & 0x7Fu) != cvt_e4m3(q)) {
             ++count;
             atomicMin(res + 1, i);
         }

@@ -174,9 +174,7 @@ __device__ __forceinline__ float amax16(const float2* p, bool hi) {
 // so that a -0 could not give the byte 0x80.
 template <bool G1>
 __device__ __forceinline__ void block_scale(float a, float g, const float* inv_tab, uint32_t& s, float& inv) {
-    const float r6 = __uint_as_float(0x3E2AAAABu);  // fl(1/6)
-    const float q0 = __fmul_rn(a, r6);
-    float t = __fmaf_rn(__fmaf_rn(-6.0f, q0, a), r6, q0);
+    float t = div6_refined(a);
     if (!G1) t = __fdiv_rn(t, g);
     s = cvt_e4m3(t) & 0x7Fu;
     if (G1) {

@@ -393,20 +393,25 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
     return h & 0xFF;
 }
 
-// fl(a / 6) for finite a >= 0 without a divide instruction: q0 = fl(a * fl(1/6)),
-// then one refinement with the exact remainder a - 6 q0 (an FMA), the
-// division-by-a-constant step of Markstein ("IA-64 and Elementary
-// Functions", 2000) and Brisebarre, Muller and Raina (IEEE Trans. Computers,
-// 2004).  fp4attn_probe_div6 checks it bit for bit against the IEEE quotient
-// for every non-negative finite fp32 value.  Below 2^-123 the quotient (or a
-// itself) is subnormal, the product a * fl(1/6) loses bits and the refinement
-// is not exact: those a take the IEEE divide.
-__device__ __forceinline__ float div6_rn(float a) {
-    if (__builtin_expect(a < __uint_as_float(0x02000000u), 0)) return __fdiv_rn(a, 6.0f);  // 2^-123
+// fl(a / 6) for finite a >= 2^-123 without a divide instruction:
+// q0 = fl(a * fl(1/6)), then one refinement with the exact remainder
+// a - 6 q0 (an FMA), the division-by-a-constant step of Markstein ("IA-64 and
+// Elementary Functions", 2000) and Brisebarre, Muller and Raina (IEEE Trans.
+// Computers, 2004).  Below 2^-123 the quotient (or a itself) is subnormal, the
+// product a * fl(1/6) loses bits and the refinement is not exact; the result
+// is then still a non-negative value below 2^-125.
+__device__ __forceinline__ float div6_refined(float a) {
     const float r6 = __uint_as_float(0x3E2AAAABu);  // fl(1/6)
     const float q0 = __fmul_rn(a, r6);
-    const float rem = __fmaf_rn(-6.0f, q0, a);
-    return __fmaf_rn(rem, r6, q0);
+    return __fmaf_rn(__fmaf_rn(-6.0f, q0, a), r6, q0);
+}
+
+// fl(a / 6) for every finite a >= 0: the refined quotient, and the IEEE divide
+// below 2^-123.  fp4attn_probe_div6 checks it bit for bit against the IEEE
+// quotient for every non-negative finite fp32 value.
+__device__ __forceinline__ float div6_rn(float a) {
+    if (__builtin_expect(a < __uint_as_float(0x02000000u), 0)) return __fdiv_rn(a, 6.0f);  // 2^-123
+    return div6_refined(a);
 }
 
 // Value of a UE4M3 byte (exact).

@@ -23,8 +23,10 @@ def assert_prologue_equal(g, o, what):
 
 
 def test_block_scale_quotient_is_the_ieee_quotient_for_every_input():
-    """The prologue computes amax / 6 with a multiply and an FMA refinement;
-    every non-negative finite fp32 amax gives the IEEE quotient's bits."""
+    """amax / 6 by a multiply and an FMA refinement: with the IEEE divide
+    below 2^-123 every non-negative finite fp32 amax gives the IEEE
+    quotient's bits, and without it (the prologue's block scale) every amax
+    gives the UE4M3 byte of the IEEE quotient."""
     count, first = fa().fp4attn_probe_div6()
     assert count == 0, f"{count} mismatches, first at bits {first:#010x}"
 
