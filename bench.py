@@ -61,8 +61,8 @@ ATTN_TRAFFIC_BYTES = {
     ("5e2fc71fa917c49f", "clip15s"): 6 * (0.4297e9 + 0.2081e9),
 }
 PROLOGUE_TRAFFIC_BYTES = {
-    ("6fdcbc5216d99518", "clip15s_8heads"): 0.5985e9 + 0.0753e9,
-    ("6fdcbc5216d99518", "clip15s"): 6 * (0.5985e9 + 0.0753e9),
+    ("37e1301caa52c2b6", "clip15s_8heads"): 0.5990e9 + 0.0756e9,
+    ("37e1301caa52c2b6", "clip15s"): 6 * (0.5990e9 + 0.0756e9),
 }
 
 
