@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -51,18 +52,19 @@ PAGES_CONTEXT = {
     "fused_transform": {"value": "under 1 ms per attention call", "hardware": "GB200"},
 }
 # ncu DRAM bytes (read + write) per launch, keyed by the sha256 prefix of the
-# kernel source they were measured on and the workload; a changed kernel reports
-# null until it is profiled again (profiles/ holds the commands).  The 15-second
+# kernel source they were measured on (comments and blank space removed) and
+# the workload; a changed kernel reports null until it is profiled again
+# (profiles/ holds the commands).  The 15-second
 # clip's figures are the eight-head capture (clip15s_8heads, the same head
 # length, a few GB on the device) times six: heads are independent and the
 # traffic of a launch grows with their number.
 ATTN_TRAFFIC_BYTES = {
-    ("5e2fc71fa917c49f", "clip15s_8heads"): 0.4297e9 + 0.2081e9,
-    ("5e2fc71fa917c49f", "clip15s"): 6 * (0.4297e9 + 0.2081e9),
+    ("05cb295263156a8d", "clip15s_8heads"): 0.4297e9 + 0.2081e9,
+    ("05cb295263156a8d", "clip15s"): 6 * (0.4297e9 + 0.2081e9),
 }
 PROLOGUE_TRAFFIC_BYTES = {
-    ("37e1301caa52c2b6", "clip15s_8heads"): 0.5990e9 + 0.0756e9,
-    ("37e1301caa52c2b6", "clip15s"): 6 * (0.5990e9 + 0.0756e9),
+    ("403b668cf754852d", "clip15s_8heads"): 0.5990e9 + 0.0756e9,
+    ("403b668cf754852d", "clip15s"): 6 * (0.5990e9 + 0.0756e9),
 }
 
 
@@ -75,8 +77,15 @@ def attention_flops(B, H, N, D=128):
 
 
 def source_hash(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256 prefix of a kernel source with its comments and blank space
+    removed: the counters stay attached to the code they were taken on, not
+    to its comments."""
+    with open(path, encoding="utf-8") as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
 def measured_peaks():

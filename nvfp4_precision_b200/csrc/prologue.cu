@@ -23,7 +23,10 @@
 // (0 <= w < W) owns rows 16w..16w+15 of every tile: it waits for the slot to
 // fill, copies its rows into registers, arrives on the slot's empty barrier
 // and computes.  No CTA-wide barrier is taken after the set-up, so the
-// consumer warps drift freely within the depth of the ring.
+// consumer warps drift freely within the depth of the ring.  The producer
+// takes a ticket only when a slot is free and asks for the next run with the
+// last ticket of the current one, so a CTA holds at most NSLOT + run
+// unfinished tickets; the lead L is sized from that at launch.
 //
 // Key-sum rows: lane l sums channels 4l..4l+3 of the warp's 16 rows into four
 // int64 registers.  A warp keeps summing while its tiles stay on one head;
@@ -35,7 +38,9 @@
 // a warp that waits for a head's sums never holds any of them back.  A K row
 // needs its head's means: the consumer warp waits for the head's count to
 // reach every chunk, then computes the 128 means once per head into its own
-// shared memory.
+// shared memory.  With key sums, a warp copies its rows and releases the
+// slot before it flushes a run or waits for a head's means, so neither
+// holds up the ring.
 //
 // Q / K rows: two lanes per row.  Lane h holds the pairs (x_i, x_{i+64}) for
 // i in [32h, 32h+32) as 32 packed fp32x2 registers: the butterflies of stride
@@ -46,7 +51,9 @@
 // round-to-nearest operation in the same stage order as the plain CPU
 // definition, so the codes are bit-identical to it, signed zeros included.
 // Each lane then owns four whole 16-value blocks: per-block amax, the UE4M3
-// scale amax/6/g, E2M1 codes of y * (1/(g * scale)).
+// scale amax/6/g, E2M1 codes of y * (1/(g * scale)).  The kernel comes in one
+// instance per setting of the two transforms, and the packing in one version
+// for g == 1 (scale reciprocals from a table) and one for other g.
 //
 // Dynamic global scales (g = amax / (6*448) of each whole transformed tensor)
 // take two launches of the same kernel: the first (AMAX) does the key sums and
