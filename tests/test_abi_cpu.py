@@ -88,6 +88,16 @@ def test_forward_validation_before_launch(fa):
 def test_probe_validation(fa):
     assert fa.lib.fp4attn_probe_qk_tile(None, None, None, None, None, None) == fa.ERR_INVALID_ARG
     assert fa.lib.fp4attn_probe_wait_timeout(None, 1000, None) == fa.ERR_INVALID_ARG
+    # the tensor-core rate probe: mode, repetition count and pointers are
+    # checked before any CUDA call
+    word = ctypes.c_int64(0)
+    status = ctypes.c_int32(0)
+    p64, p32 = ctypes.cast(ctypes.pointer(word), ctypes.c_void_p), ctypes.cast(ctypes.pointer(status), ctypes.c_void_p)
+    assert fa.lib.fp4attn_probe_mma_rate(2, 10, p64, p32, None) == fa.ERR_INVALID_ARG
+    assert fa.lib.fp4attn_probe_mma_rate(0, 0, p64, p32, None) == fa.ERR_INVALID_ARG
+    assert fa.lib.fp4attn_probe_mma_rate(1, 1000001, p64, p32, None) == fa.ERR_INVALID_ARG
+    assert fa.lib.fp4attn_probe_mma_rate(0, 10, None, p32, None) == fa.ERR_INVALID_ARG
+    assert fa.lib.fp4attn_probe_mma_rate(0, 10, p64, None, None) == fa.ERR_INVALID_ARG
     assert fa.lib.fp4attn_encode_f32(None, 5, None, None, None) == fa.ERR_INVALID_ARG
 
 
